@@ -1,0 +1,28 @@
+"""B200-native (sm_100a) per-rank hot path of context-parallel attention.
+
+* ``fwd``       non-causal attention with LSE (tcgen05 / TMEM / TMA kernel for bf16)
+* ``merge``     exact (O, LSE) merge of two key-chunk partials (Ring Attention step)
+* ``seq2head``  Ulysses sequence shards -> head groups over P virtual ranks
+* ``head2seq``  the inverse permute
+* ``ring_attention`` / ``ulysses_attention``  the two per-rank compositions
+
+All compute runs in ``libcpattn.so`` (C ABI in ``include/cpattn.h``); this package only
+marshals arguments.  ``workloads`` holds the seeded synthetic inputs.
+"""
+
+from ._binding import (  # noqa: F401
+    BF16,
+    F32,
+    CpattnError,
+    device_error,
+    fwd,
+    head2seq,
+    lib,
+    library_path,
+    merge,
+    selftest_wait_timeout,
+    seq2head,
+    status_str,
+    version,
+)
+from .paths import ring_attention, ulysses_attention  # noqa: F401

@@ -1,0 +1,181 @@
+"""ctypes binding of libcpattn.so (include/cpattn.h).  Argument marshalling only: every
+step of the path runs in the library's CUDA kernels.  PyTorch provides device memory and
+the current stream; nothing here computes on the host.  There is no fallback: if the
+library is missing or a call fails, an exception is raised.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libcpattn.so")
+
+BF16, F32 = 0, 1
+OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_CUDA, ERR_DEVICE_TIMEOUT = range(7)
+
+_lock = threading.Lock()
+_lib = None
+
+
+class CpattnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_str(status)}")
+
+
+def library_path() -> str:
+    return LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """Load libcpattn.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with "
+                    "`python -m context_long_sequence_non_b200.build` (no CPU fallback exists)")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, i, f, ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong
+            L.cpattn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+            L.cpattn_merge.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
+            L.cpattn_seq2head.argtypes = [vp, vp, i, i, i, i, i, vp]
+            L.cpattn_head2seq.argtypes = [vp, vp, i, i, i, i, i, vp]
+            L.cpattn_status_str.argtypes = [i]
+            L.cpattn_status_str.restype = ctypes.c_char_p
+            L.cpattn_device_error.argtypes = []
+            L.cpattn_selftest_wait_timeout.argtypes = [ll, vp]
+            L.cpattn_version.argtypes = []
+            for name in ("cpattn_fwd", "cpattn_merge", "cpattn_seq2head", "cpattn_head2seq",
+                         "cpattn_device_error", "cpattn_selftest_wait_timeout", "cpattn_version"):
+                getattr(L, name).restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+def status_str(status: int) -> str:
+    return lib().cpattn_status_str(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise CpattnError(status, what)
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return BF16
+    if t == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("tensors must live on a CUDA device")
+            if not t.is_contiguous():
+                raise ValueError("tensors must be contiguous")
+
+
+def fwd(q, k, v, out=None, lse=None, scale=None, out_dtype=None, want_lse=True, stream=None):
+    """Non-causal attention ``softmax(scale * Q K^T) V`` with its log-sum-exp.
+
+    q: [B][Sq][H][D], k/v: [B][Skv][H][D] (bf16 -> tcgen05 kernel, fp32 -> CUDA-core
+    kernel).  Returns ``(out [B][Sq][H][D], lse [B][H][Sq] float32)``.
+    """
+    B, Sq, H, D = q.shape
+    Skv = k.shape[1]
+    if k.shape != (B, Skv, H, D) or v.shape != (B, Skv, H, D):
+        raise ValueError("k and v must be [B][Skv][H][D] matching q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out_dtype is None:
+        out_dtype = q.dtype
+    if out is None:
+        out = torch.empty((B, Sq, H, D), dtype=out_dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    _need_cuda(q, k, v, out, lse)
+    st = lib().cpattn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Sq, Skv, D,
+                          float(scale), _dtype_code(q.dtype), _dtype_code(out.dtype),
+                          _stream(stream))
+    _check(st, "cpattn_fwd")
+    return out, lse
+
+
+def merge(o_a, lse_a, o_b, lse_b, out=None, lse=None, stream=None):
+    """Exact merge of two partial (O, LSE) results; ``out``/``lse`` may be o_a/lse_a."""
+    B, S, H, D = o_a.shape
+    if out is None:
+        out = torch.empty_like(o_a)
+    if lse is None:
+        lse = torch.empty_like(lse_a)
+    _need_cuda(o_a, lse_a, o_b, lse_b, out, lse)
+    st = lib().cpattn_merge(_ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b), _ptr(out), _ptr(lse),
+                            B, H, S, D, _dtype_code(o_a.dtype), _stream(stream))
+    _check(st, "cpattn_merge")
+    return out, lse
+
+
+def seq2head(src, P, out=None, stream=None):
+    """[P][S_l][H][D] sequence shards -> [P][P*S_l][H/P][D] head groups (bit copy)."""
+    P_, S_l, H, D = src.shape
+    if P_ != P:
+        raise ValueError("src.shape[0] must equal P")
+    if out is None:
+        out = torch.empty((P, P * S_l, H // P, D), dtype=src.dtype, device=src.device)
+    _need_cuda(src, out)
+    st = lib().cpattn_seq2head(_ptr(src), _ptr(out), P, S_l, H, D, src.element_size(),
+                               _stream(stream))
+    _check(st, "cpattn_seq2head")
+    return out
+
+
+def head2seq(src, P, out=None, stream=None):
+    """[P][P*S_l][Hp][D] head groups -> [P][S_l][P*Hp][D] sequence shards (bit copy)."""
+    P_, S_full, Hp, D = src.shape
+    if P_ != P or S_full % P:
+        raise ValueError("src must be [P][P*S_l][Hp][D]")
+    S_l, H = S_full // P, Hp * P
+    if out is None:
+        out = torch.empty((P, S_l, H, D), dtype=src.dtype, device=src.device)
+    _need_cuda(src, out)
+    st = lib().cpattn_head2seq(_ptr(src), _ptr(out), P, S_l, H, D, src.element_size(),
+                               _stream(stream))
+    _check(st, "cpattn_head2seq")
+    return out
+
+
+def device_error() -> int:
+    """Synchronize and read/clear the device error word (OK or ERR_DEVICE_TIMEOUT)."""
+    return lib().cpattn_device_error()
+
+
+def selftest_wait_timeout(limit_cycles: int, stream=None):
+    _check(lib().cpattn_selftest_wait_timeout(int(limit_cycles), _stream(stream)),
+           "cpattn_selftest_wait_timeout")
+
+
+def version() -> int:
+    return lib().cpattn_version()

@@ -1,0 +1,209 @@
+// api.cu -- the C ABI of include/cpattn.h: host-side argument checks, TMA tensor-map
+// encoding, dispatch to the kernels, and the per-device error word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "cpattn.h"
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace {
+
+// One word per device; kernels record bounded-wait timeouts here (atomicOr).
+__device__ int g_cpattn_err;
+
+constexpr int kMaxDevices = 64;
+
+int* device_error_word() {
+  static int* addr[kMaxDevices] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_cpattn_err) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<int*>(p);
+  }
+  return addr[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// [B][S][H][D] bf16 tensor, box = 64 head-dim columns x 1 head x 128 tokens x 1 batch,
+// 128-byte swizzle (the layout tcgen05 reads through a 128-byte-swizzle descriptor).
+bool encode_bshd_bf16(CUtensorMap* map, const void* ptr, int B, int S, int H, int D) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(S), cuuint64_t(B)};
+  const cuuint64_t strides[3] = {cuuint64_t(D) * 2, cuuint64_t(H) * D * 2,
+                                 cuuint64_t(S) * H * D * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA; }
+
+int elem_size(int dtype) { return dtype == CPATTN_BF16 ? 2 : (dtype == CPATTN_F32 ? 4 : 0); }
+
+}  // namespace
+
+extern "C" {
+
+int cpattn_version(void) { return (1 << 16) | 0; }
+
+const char* cpattn_status_str(int status) {
+  switch (status) {
+    case CPATTN_OK: return "CPATTN_OK";
+    case CPATTN_ERR_NULL: return "CPATTN_ERR_NULL: a required pointer is NULL";
+    case CPATTN_ERR_SHAPE: return "CPATTN_ERR_SHAPE: a size is out of range or inconsistent";
+    case CPATTN_ERR_ALIGN: return "CPATTN_ERR_ALIGN: a pointer is not suitably aligned";
+    case CPATTN_ERR_UNSUPPORTED: return "CPATTN_ERR_UNSUPPORTED: no kernel for this dtype/size";
+    case CPATTN_ERR_CUDA: return "CPATTN_ERR_CUDA: a CUDA call or kernel launch failed";
+    case CPATTN_ERR_DEVICE_TIMEOUT:
+      return "CPATTN_ERR_DEVICE_TIMEOUT: a kernel's bounded wait ran out";
+    default: return "CPATTN: unknown status";
+  }
+}
+
+int cpattn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
+               int Sq, int Skv, int D, float scale, int in_dtype, int out_dtype,
+               cpattn_stream_t stream) {
+  if (B < 1 || H < 1 || Sq < 1 || Skv < 0 || D < 1) return CPATTN_ERR_SHAPE;
+  if (!(std::isfinite(scale) && scale > 0.f)) return CPATTN_ERR_SHAPE;
+  const int in_es = elem_size(in_dtype), out_es = elem_size(out_dtype);
+  if (in_es == 0 || out_es == 0) return CPATTN_ERR_UNSUPPORTED;
+  if (q == nullptr || out == nullptr) return CPATTN_ERR_NULL;
+  if (Skv > 0 && (k == nullptr || v == nullptr)) return CPATTN_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(out, 16) || (Skv > 0 && (!aligned(k, 16) || !aligned(v, 16))) ||
+      (lse != nullptr && !aligned(lse, 4)))
+    return CPATTN_ERR_ALIGN;
+  if (in_dtype == CPATTN_BF16 && D != 64 && D != 128) return CPATTN_ERR_UNSUPPORTED;
+  if (in_dtype == CPATTN_F32 && D > 256) return CPATTN_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535) return CPATTN_ERR_SHAPE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t out_bytes = size_t(B) * Sq * H * D * out_es;
+  if (Skv == 0) {
+    if (out_bytes % 16 != 0) return CPATTN_ERR_SHAPE;
+    return cuda_status(cpattn::launch_fill_empty(out, out_bytes, lse, size_t(B) * H * Sq, st));
+  }
+  if (in_dtype == CPATTN_BF16) {
+    int* err = device_error_word();
+    if (err == nullptr) return CPATTN_ERR_CUDA;
+    CUtensorMap tq, tk, tv;
+    if (!encode_bshd_bf16(&tq, q, B, Sq, H, D) || !encode_bshd_bf16(&tk, k, B, Skv, H, D) ||
+        !encode_bshd_bf16(&tv, v, B, Skv, H, D))
+      return CPATTN_ERR_CUDA;
+    const float scale_log2 = float(double(scale) * 1.4426950408889634074);
+    return cuda_status(cpattn::launch_attn_fwd_sm100(tq, tk, tv, out, lse, B, H, Sq, Skv, D,
+                                                     scale_log2, out_dtype == CPATTN_F32, err,
+                                                     cpattn::kDefaultWaitLimit, st));
+  }
+  // fp32 inputs: CUDA-core kernel
+  return cuda_status(cpattn::launch_attn_fwd_f32(
+      static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+      out, lse, B, H, Sq, Skv, D, scale, out_dtype == CPATTN_BF16, st));
+}
+
+int cpattn_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b, void* o,
+                 float* lse, int B, int H, int S, int D, int dtype, cpattn_stream_t stream) {
+  if (B < 1 || H < 1 || S < 1 || D < 1) return CPATTN_ERR_SHAPE;
+  const int es = elem_size(dtype);
+  if (es == 0) return CPATTN_ERR_UNSUPPORTED;
+  if ((D * es) % 16 != 0) return CPATTN_ERR_SHAPE;
+  if (!o_a || !lse_a || !o_b || !lse_b || !o || !lse) return CPATTN_ERR_NULL;
+  if (!aligned(o_a, 16) || !aligned(o_b, 16) || !aligned(o, 16) || !aligned(lse_a, 4) ||
+      !aligned(lse_b, 4) || !aligned(lse, 4))
+    return CPATTN_ERR_ALIGN;
+  const size_t ob = size_t(B) * S * H * D * es, lb = size_t(B) * H * S * 4;
+  // o may be o_a exactly (in-place accumulate); any other overlap would race
+  if ((o != o_a && overlap(o, ob, o_a, ob)) || overlap(o, ob, o_b, ob) ||
+      (lse != lse_a && overlap(lse, lb, lse_a, lb)) || overlap(lse, lb, lse_b, lb))
+    return CPATTN_ERR_SHAPE;
+  return cuda_status(cpattn::launch_merge(o_a, lse_a, o_b, lse_b, o, lse, B, H, S, D, es,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static int permute_args(const void* src, void* dst, int P, int S_local, int H, int D,
+                        int elem_bytes, long long* run_vec) {
+  if (P < 1 || S_local < 1 || H < 1 || D < 1) return CPATTN_ERR_SHAPE;
+  if (elem_bytes != 2 && elem_bytes != 4) return CPATTN_ERR_SHAPE;
+  if (H % P != 0) return CPATTN_ERR_SHAPE;
+  const long long run_bytes = (long long)(H / P) * D * elem_bytes;
+  if (run_bytes % 16 != 0) return CPATTN_ERR_SHAPE;
+  if ((long long)P * P * S_local > 0x7fffffffLL || run_bytes / 16 > 0x7fffffffLL)
+    return CPATTN_ERR_SHAPE;
+  if (src == nullptr || dst == nullptr) return CPATTN_ERR_NULL;
+  if (!aligned(src, 16) || !aligned(dst, 16)) return CPATTN_ERR_ALIGN;
+  const size_t bytes = size_t(P) * S_local * H * D * elem_bytes;
+  if (overlap(src, bytes, dst, bytes)) return CPATTN_ERR_SHAPE;
+  *run_vec = run_bytes / 16;
+  return CPATTN_OK;
+}
+
+int cpattn_seq2head(const void* src, void* dst, int P, int S_local, int H, int D, int elem_bytes,
+                    cpattn_stream_t stream) {
+  long long run_vec = 0;
+  const int st = permute_args(src, dst, P, S_local, H, D, elem_bytes, &run_vec);
+  if (st != CPATTN_OK) return st;
+  return cuda_status(cpattn::launch_seq2head(src, dst, P, S_local, run_vec,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int cpattn_head2seq(const void* src, void* dst, int P, int S_local, int H, int D, int elem_bytes,
+                    cpattn_stream_t stream) {
+  long long run_vec = 0;
+  const int st = permute_args(src, dst, P, S_local, H, D, elem_bytes, &run_vec);
+  if (st != CPATTN_OK) return st;
+  return cuda_status(cpattn::launch_head2seq(src, dst, P, S_local, run_vec,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int cpattn_device_error(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return CPATTN_ERR_CUDA;
+  int* addr = device_error_word();
+  if (addr == nullptr) return CPATTN_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_cpattn_err, sizeof(int)) != cudaSuccess) return CPATTN_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_cpattn_err, &zero, sizeof(int)) != cudaSuccess) return CPATTN_ERR_CUDA;
+  return (word & cpattn::kDevErrTimeout) ? CPATTN_ERR_DEVICE_TIMEOUT : CPATTN_OK;
+}
+
+int cpattn_selftest_wait_timeout(long long limit_cycles, cpattn_stream_t stream) {
+  if (limit_cycles < 1 || limit_cycles > (1LL << 31)) return CPATTN_ERR_SHAPE;
+  int* err = device_error_word();
+  if (err == nullptr) return CPATTN_ERR_CUDA;
+  return cuda_status(cpattn::launch_wait_timeout_selftest(err, limit_cycles,
+                                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,399 @@
+// attn_sm100.cu -- non-causal attention forward on B200 tensor cores (tcgen05 + TMEM + TMA).
+//
+// What it computes (AllGather KV / 环形注意力 Ring Attention sections of "Scaling AI
+// Inference Across Multiple GPUs Using NVIDIA TensorRT with Multi-Device Inference
+// Support", Figs. 2-3): for every (b, h, query row i)
+//   O_i = sum_j softmax_j(scale * q_i . k_j) v_j,   LSE_i = ln sum_j exp(scale * q_i . k_j)
+// streamed over 128-key blocks with an online softmax, so that the (O, LSE) of separate
+// key chunks merge exactly afterwards (the Ring Attention step).
+//
+// Design (one CTA = 256 query rows of one (b, h), 12 warps):
+//   warps 0-3  softmax for Q tile 0  (TMEM lanes 0..127, one thread per query row)
+//   warps 4-7  softmax for Q tile 1
+//   warp  8    TMA producer: Q0, Q1 once, then K_0, V_0, K_1, V_1, ... into a 4-slot ring
+//   warp  9    TMEM allocator + single-thread tcgen05.mma issuer
+// TMEM (512 columns): S0 | S1 (128 fp32 columns each; P_i is written back over S_i as
+// bf16 pairs) | O0 | O1 (D fp32 columns each).  S = Q K^T runs smem x smem; O += P V
+// takes P from TMEM and V from smem (MN-major).  While softmax works on one Q tile the
+// tensor core runs the other tile's MMAs (ping-pong), and TMA prefetches ahead.
+// Softmax works in base 2: x = s * scale * log2(e); the running max is only raised when
+// it grows by more than kRescaleLog2 (a stale max is exact because the final
+// normalisation uses the same max); O is rescaled in TMEM by the softmax warps then.
+// Every wait is bounded (mbar_wait): a stalled pipeline sets the device error word and
+// the CTA drains and exits instead of hanging.
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace cpattn {
+namespace {
+
+constexpr int kBlockM = 128;     // query rows per Q tile = TMEM lanes
+constexpr int kBlockN = 128;     // keys per K/V tile
+constexpr int kSlots = 4;        // K/V ring slots (K_j and V_j alternate)
+constexpr int kThreads = 384;
+constexpr int kWarpProducer = 8;
+constexpr int kWarpMma = 9;
+constexpr float kRescaleLog2 = 8.0f;  // raise the running max only past a 2^8 growth
+constexpr uint32_t kTmemCols = 512;
+
+template <int D>
+struct Geometry {
+  static constexpr int kBox = 64;                       // bf16 columns per TMA box (128 B)
+  static constexpr int kBoxBytes = kBlockN * kBox * 2;  // 16 KB: 128 rows x 128 B
+  static constexpr int kBoxes = D / kBox;
+  static constexpr int kTileBytes = kBoxes * kBoxBytes; // one 128-row tile of Q, K or V
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffSlots = 2 * kTileBytes;
+  static constexpr int kBytes = kOffSlots + kSlots * kTileBytes;
+  // + slack for 1024-B alignment; never below 120 KB so that one CTA, which takes all
+  // 512 TMEM columns, is the only one resident on its SM
+  static constexpr int kDynSmem = (kBytes + 1024) > 120 * 1024 ? (kBytes + 1024) : 120 * 1024;
+};
+
+struct __align__(8) Barriers {
+  uint64_t q_full;
+  uint64_t full[kSlots];
+  uint64_t empty[kSlots];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_full;
+  uint64_t drain;
+};
+
+template <int D, bool kOutF32>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                          const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, void* __restrict__ out,
+                          float* __restrict__ lse, int H, int Sq, int Skv, float scale_log2,
+                          int* err, long long wait_limit) {
+  using G = Geometry<D>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ Barriers bars;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t smem_base = smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int q_first = blockIdx.x * (2 * kBlockM);
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int n_kv = (Skv + kBlockN - 1) / kBlockN;
+  volatile int* abort_flag = &abort_sh;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars.q_full), 1);
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(smem_u32(&bars.full[s]), 1);
+      mbar_init(smem_u32(&bars.empty[s]), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(smem_u32(&bars.s_full[t]), 1);
+      mbar_init(smem_u32(&bars.p_full[t]), kBlockM);
+    }
+    mbar_init(smem_u32(&bars.o_full), 1);
+    mbar_init(smem_u32(&bars.drain), 1);
+    abort_sh = 0;
+    fence_mbar_init();
+  }
+  if (warp == kWarpProducer && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(smem_u32(&tmem_base_sh), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp < 8) {
+    // ------------------------------------------------------------------ softmax warps
+    const int tile = warp >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;  // row within the Q tile == TMEM lane
+    const uint32_t lane_bits = uint32_t(quarter * 32) << 16;
+    const uint32_t t_s = tmem + lane_bits + uint32_t(tile * kBlockN);
+    const uint32_t t_o = tmem + lane_bits + uint32_t(2 * kBlockN + tile * D);
+    const uint32_t bar_s = smem_u32(&bars.s_full[tile]);
+    const uint32_t bar_p = smem_u32(&bars.p_full[tile]);
+    float m = -INFINITY;  // running (possibly stale) max of x = s * scale * log2(e)
+    float l = 0.f;        // running sum of 2^(x - m)
+    bool ok = true;
+
+    for (int j = 0; j < n_kv; ++j) {
+      ok = mbar_wait(bar_s, j & 1, abort_flag, err, wait_limit);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+
+      float x[kBlockN];
+#pragma unroll
+      for (int c = 0; c < kBlockN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(t_s + c * 32, r);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(r[e]);
+      }
+      const int valid = Skv - j * kBlockN;  // keys of this tile inside the sequence
+      if (valid < kBlockN) {
+#pragma unroll
+        for (int c = 0; c < kBlockN; ++c)
+          if (c >= valid) x[c] = -INFINITY;
+      }
+      // row maximum of the scaled logits (scale > 0 is a precondition of the call)
+      float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
+#pragma unroll
+      for (int c = 4; c < kBlockN; c += 4) {
+        mx0 = fmaxf(mx0, x[c]); mx1 = fmaxf(mx1, x[c + 1]);
+        mx2 = fmaxf(mx2, x[c + 2]); mx3 = fmaxf(mx3, x[c + 3]);
+      }
+      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * scale_log2;
+      float alpha = 1.0f;
+      bool rescale = false;
+      if (j == 0) {
+        m = m_tile;
+      } else {
+        const bool grow = m_tile > m + kRescaleLog2;
+        rescale = __any_sync(0xffffffffu, grow);
+        if (rescale) {
+          const float m_new = grow ? m_tile : m;
+          alpha = ex2(m - m_new);
+          m = m_new;
+          l *= alpha;
+        }
+      }
+      // p = 2^(x - m), rounded to bf16 for the PV product, written over S as bf16 pairs
+      const float neg_m = -m;
+      float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float p0 = ex2(fmaf(x[half * 64 + 2 * e], scale_log2, neg_m));
+          const float p1 = ex2(fmaf(x[half * 64 + 2 * e + 1], scale_log2, neg_m));
+          sum0 += p0;
+          sum1 += p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(t_s + half * 32, pk);
+      }
+      l += sum0 + sum1;
+      if (rescale) {
+        // rescale this warp's O rows by alpha: PV of the previous block has completed
+        // (the issuer committed this block's S after it) and the next PV waits for
+        // p_full, so nothing else touches O now
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(t_o + c * 32, r);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st32(t_o + c * 32, r);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_p);
+    }
+
+    // ------------------------------------------------------------------ epilogue
+    if (ok) {
+      ok = mbar_wait(smem_u32(&bars.o_full), 0, abort_flag, err, wait_limit);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      const int q = q_first + tile * kBlockM + row;
+      const bool in_range = q < Sq;
+      const float inv_l = 1.0f / l;
+      const size_t row_off = ((size_t(b) * Sq + (in_range ? q : 0)) * H + h) * size_t(D);
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(t_o + c * 32, r);
+        if (in_range) {
+          if constexpr (kOutF32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + row_off + c * 32);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(r[4 * e]) * inv_l,
+                                   __uint_as_float(r[4 * e + 1]) * inv_l,
+                                   __uint_as_float(r[4 * e + 2]) * inv_l,
+                                   __uint_as_float(r[4 * e + 3]) * inv_l);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + row_off + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              uint4 v;
+              v.x = pack_bf16x2(__uint_as_float(r[8 * e + 0]) * inv_l, __uint_as_float(r[8 * e + 1]) * inv_l);
+              v.y = pack_bf16x2(__uint_as_float(r[8 * e + 2]) * inv_l, __uint_as_float(r[8 * e + 3]) * inv_l);
+              v.z = pack_bf16x2(__uint_as_float(r[8 * e + 4]) * inv_l, __uint_as_float(r[8 * e + 5]) * inv_l);
+              v.w = pack_bf16x2(__uint_as_float(r[8 * e + 6]) * inv_l, __uint_as_float(r[8 * e + 7]) * inv_l);
+              dst[e] = v;
+            }
+          }
+        }
+      }
+      if (in_range && lse != nullptr) {
+        // LSE = ln(2^m * l) = (m + log2 l) * ln 2
+        lse[(size_t(b) * H + h) * Sq + q] = (m + log2f(l)) * 0.69314718055994530942f;
+      }
+    }
+  } else if (warp == kWarpProducer) {
+    // ------------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      const uint32_t bar_q = smem_u32(&bars.q_full);
+      mbar_arrive_expect_tx(bar_q, 2 * G::kTileBytes);
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int bx = 0; bx < G::kBoxes; ++bx)
+          tma_load_4d(smem_base + G::kOffQ + t * G::kTileBytes + bx * G::kBoxBytes, &tm_q, bar_q,
+                      bx * G::kBox, h, q_first + t * kBlockM, b);
+      int issued = 0;
+      for (int use = 0; use < 2 * n_kv; ++use) {
+        const int slot = use % kSlots;
+        const uint32_t ph = uint32_t(use / kSlots) & 1u;
+        if (!mbar_wait(smem_u32(&bars.empty[slot]), ph ^ 1u, abort_flag, err, wait_limit)) break;
+        const uint32_t bar_f = smem_u32(&bars.full[slot]);
+        mbar_arrive_expect_tx(bar_f, G::kTileBytes);
+        const CUtensorMap* map = (use & 1) ? &tm_v : &tm_k;
+        const int key0 = (use >> 1) * kBlockN;
+#pragma unroll
+        for (int bx = 0; bx < G::kBoxes; ++bx)
+          tma_load_4d(smem_base + G::kOffSlots + slot * G::kTileBytes + bx * G::kBoxBytes, map,
+                      bar_f, bx * G::kBox, h, key0, b);
+        issued = use + 1;
+      }
+      // drain: every issued copy must have landed before the CTA's shared memory is
+      // released (immediate on the normal path, where the consumer already saw them)
+      drain_wait(bar_q, 0, wait_limit);
+      for (int use = issued - kSlots < 0 ? 0 : issued - kSlots; use < issued; ++use)
+        drain_wait(smem_u32(&bars.full[use % kSlots]), uint32_t(use / kSlots) & 1u, wait_limit);
+    }
+    __syncwarp();
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, D, true);
+      const uint32_t q_addr[2] = {smem_base + G::kOffQ, smem_base + G::kOffQ + G::kTileBytes};
+      const uint32_t t_s[2] = {tmem, tmem + kBlockN};
+      const uint32_t t_o[2] = {tmem + 2 * kBlockN, tmem + 2 * kBlockN + D};
+
+      // S_t = Q_t K^T over D in K=16 steps; K-major 128-B swizzled operands: 32 B per
+      // step inside a 128-B row, the next 64 columns in the next box
+      auto issue_qk = [&](int t, uint32_t k_addr) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * G::kBoxBytes + (kk & 3) * 32;
+          mma_ss(t_s[t], sdesc_sw128(q_addr[t] + off, 16, 1024),
+                 sdesc_sw128(k_addr + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      // O_t += P_t V over the 128 keys in K=16 steps; P from TMEM (8 columns = 16 bf16
+      // per step), V MN-major: 16 key rows = 2 KB per step, the d halves one box apart
+      auto issue_pv = [&](int t, uint32_t v_addr, bool accumulate) {
+#pragma unroll
+        for (int kk = 0; kk < kBlockN / 16; ++kk) {
+          mma_ts(t_o[t], t_s[t] + kk * 8, sdesc_sw128(v_addr + kk * 16 * 128, G::kBoxBytes, 1024),
+                 idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+        }
+      };
+      auto slot_addr = [&](int use) {
+        return smem_base + G::kOffSlots + (use % kSlots) * G::kTileBytes;
+      };
+      auto wait_full = [&](int use) {
+        return mbar_wait(smem_u32(&bars.full[use % kSlots]), uint32_t(use / kSlots) & 1u,
+                         abort_flag, err, wait_limit);
+      };
+
+      bool ok = mbar_wait(smem_u32(&bars.q_full), 0, abort_flag, err, wait_limit) && wait_full(0);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0, slot_addr(0));
+        tc_commit(smem_u32(&bars.s_full[0]));
+        issue_qk(1, slot_addr(0));
+        tc_commit(smem_u32(&bars.s_full[1]));
+        tc_commit(smem_u32(&bars.empty[0]));
+      }
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int use_v = 2 * j + 1, use_k = 2 * j + 2;
+        const bool more = j + 1 < n_kv;
+        if (!(ok = wait_full(use_v))) break;
+        if (!(ok = mbar_wait(smem_u32(&bars.p_full[0]), j & 1, abort_flag, err, wait_limit))) break;
+        tc_fence_after();
+        issue_pv(0, slot_addr(use_v), j > 0);
+        if (more) {
+          if (!(ok = wait_full(use_k))) break;
+          tc_fence_after();
+          issue_qk(0, slot_addr(use_k));
+          tc_commit(smem_u32(&bars.s_full[0]));
+        }
+        if (!(ok = mbar_wait(smem_u32(&bars.p_full[1]), j & 1, abort_flag, err, wait_limit))) break;
+        tc_fence_after();
+        issue_pv(1, slot_addr(use_v), j > 0);
+        tc_commit(smem_u32(&bars.empty[use_v % kSlots]));
+        if (more) {
+          issue_qk(1, slot_addr(use_k));
+          tc_commit(smem_u32(&bars.s_full[1]));
+          tc_commit(smem_u32(&bars.empty[use_k % kSlots]));
+        }
+      }
+      if (ok) tc_commit(smem_u32(&bars.o_full));
+      // drain: no MMA may still be writing TMEM when it is freed
+      tc_commit(smem_u32(&bars.drain));
+      drain_wait(smem_u32(&bars.drain), 0, wait_limit);
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kWarpMma) tmem_dealloc(tmem, kTmemCols);
+}
+
+template <int D, bool kOutF32>
+cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* out,
+                   float* lse, int B, int H, int Sq, int Skv, float scale_log2, int* err,
+                   long long wait_limit, cudaStream_t stream) {
+  using G = Geometry<D>;
+  auto kernel = attn_fwd_sm100_kernel<D, kOutF32>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       G::kDynSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((Sq + 2 * kBlockM - 1) / (2 * kBlockM), H, B);
+  kernel<<<grid, kThreads, G::kDynSmem, stream>>>(tq, tk, tv, out, lse, H, Sq, Skv, scale_log2,
+                                                   err, wait_limit);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
+                                  const CUtensorMap& tv, void* out, float* lse, int B, int H,
+                                  int Sq, int Skv, int D, float scale_log2, bool out_f32, int* err,
+                                  long long wait_limit, cudaStream_t stream) {
+  if (D == 128) {
+    return out_f32 ? launch<128, true>(tq, tk, tv, out, lse, B, H, Sq, Skv, scale_log2, err,
+                                       wait_limit, stream)
+                   : launch<128, false>(tq, tk, tv, out, lse, B, H, Sq, Skv, scale_log2, err,
+                                        wait_limit, stream);
+  }
+  return out_f32 ? launch<64, true>(tq, tk, tv, out, lse, B, H, Sq, Skv, scale_log2, err,
+                                    wait_limit, stream)
+                 : launch<64, false>(tq, tk, tv, out, lse, B, H, Sq, Skv, scale_log2, err,
+                                     wait_limit, stream);
+}
+
+}  // namespace cpattn

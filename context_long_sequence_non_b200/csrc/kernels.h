@@ -1,0 +1,45 @@
+// kernels.h -- internal launchers behind the C ABI (include/cpattn.h).  Each returns the
+// CUDA error of its launch; argument validation happens in api.cu before any of them runs.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace cpattn {
+
+// Default bounded-wait limit in SM clock cycles (about one second at 1.9 GHz).
+constexpr long long kDefaultWaitLimit = 2000000000LL;
+
+// tcgen05 attention, bf16 in, D in {64, 128}; tensor maps describe [B][S][H][D] bf16
+// tensors with a 64 x 1 x 128 x 1 box and 128-byte swizzle.
+cudaError_t launch_attn_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
+                                  const CUtensorMap& tv, void* out, float* lse, int B, int H,
+                                  int Sq, int Skv, int D, float scale_log2, bool out_f32, int* err,
+                                  long long wait_limit, cudaStream_t stream);
+
+// fp32 CUDA-core attention, D <= 256.
+cudaError_t launch_attn_fwd_f32(const float* q, const float* k, const float* v, void* out,
+                                float* lse, int B, int H, int Sq, int Skv, int D, float scale,
+                                bool out_bf16, cudaStream_t stream);
+
+// out = 0 and lse = -inf (the empty key set).
+cudaError_t launch_fill_empty(void* out, size_t out_bytes, float* lse, size_t n_lse,
+                              cudaStream_t stream);
+
+// (O, LSE) merge; elem_bytes 2 (bf16) or 4 (f32).
+cudaError_t launch_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
+                         void* o, float* lse, int B, int H, int S, int D, int elem_bytes,
+                         cudaStream_t stream);
+
+// Ulysses permutes over 16-byte words; `run_vec` = Hp*D*elem_bytes/16.
+cudaError_t launch_seq2head(const void* src, void* dst, int P, int S_local, long long run_vec,
+                            cudaStream_t stream);
+cudaError_t launch_head2seq(const void* src, void* dst, int P, int S_local, long long run_vec,
+                            cudaStream_t stream);
+
+// One CTA waiting on an mbarrier nothing completes, with the attention kernel's bounded wait.
+cudaError_t launch_wait_timeout_selftest(int* err, long long limit, cudaStream_t stream);
+
+int sm_count();
+
+}  // namespace cpattn

@@ -1,0 +1,362 @@
+// simt.cu -- the CUDA-core kernels of the path: fp32 attention, the (O, LSE) merge of the
+// Ring Attention step, the two Ulysses permutes, the empty-key fill and the bounded-wait
+// self-test.  Merge and permutes are HBM-bound streaming kernels: 16-byte vectors, each
+// warp moving contiguous runs, several independent loads in flight per thread, grids
+// sized in multiples of the SM count.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace cpattn {
+namespace {
+
+// ------------------------------------------------------------------ fp32 attention
+// One warp per query row (b, h, i); lane l holds q[d] for d = l, l + 32, ...  Keys are
+// visited in order with an online softmax in fp32 (natural base, expf/logf).
+template <int T>
+__global__ void __launch_bounds__(256) attn_f32_kernel(const float* __restrict__ q,
+                                                       const float* __restrict__ k,
+                                                       const float* __restrict__ v, void* out,
+                                                       float* lse, int B, int H, int Sq, int Skv,
+                                                       int D, float scale, bool out_bf16) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const long long n_rows = (long long)B * H * Sq;
+  if (row >= n_rows) return;
+  const int i = int(row % Sq);
+  const int h = int((row / Sq) % H);
+  const int b = int(row / ((long long)Sq * H));
+  float qv[T], acc[T];
+  const float* qp = q + (((long long)b * Sq + i) * H + h) * D;
+#pragma unroll
+  for (int t = 0; t < T; ++t) {
+    const int d = lane + 32 * t;
+    qv[t] = d < D ? qp[d] : 0.f;
+    acc[t] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+  for (int j = 0; j < Skv; ++j) {
+    const long long kv_off = (((long long)b * Skv + j) * H + h) * D;
+    float part = 0.f;
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+      const int d = lane + 32 * t;
+      if (d < D) part = fmaf(qv[t], k[kv_off + d], part);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) part += __shfl_down_sync(0xffffffffu, part, off);
+    const float s = __shfl_sync(0xffffffffu, part, 0) * scale;
+    if (s > m) {
+      const float corr = expf(m - s);
+      l *= corr;
+#pragma unroll
+      for (int t = 0; t < T; ++t) acc[t] *= corr;
+      m = s;
+    }
+    const float p = expf(s - m);
+    l += p;
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+      const int d = lane + 32 * t;
+      if (d < D) acc[t] = fmaf(p, v[kv_off + d], acc[t]);
+    }
+  }
+  const float inv_l = 1.0f / l;
+  const long long o_off = (((long long)b * Sq + i) * H + h) * D;
+#pragma unroll
+  for (int t = 0; t < T; ++t) {
+    const int d = lane + 32 * t;
+    if (d < D) {
+      const float o = acc[t] * inv_l;
+      if (out_bf16) {
+        static_cast<uint16_t*>(out)[o_off + d] = uint16_t(pack_bf16x2(o, 0.f) & 0xFFFFu);
+      } else {
+        static_cast<float*>(out)[o_off + d] = o;
+      }
+    }
+  }
+  if (lane == 0 && lse != nullptr) lse[((long long)b * H + h) * Sq + i] = m + logf(l);
+}
+
+// ------------------------------------------------------------------ empty key set
+__global__ void fill_empty_kernel(uint4* out, size_t n_vec, float* lse, size_t n_lse) {
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_vec; i += stride)
+    out[i] = make_uint4(0u, 0u, 0u, 0u);
+  if (lse != nullptr)
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_lse; i += stride)
+      lse[i] = -INFINITY;
+}
+
+// ------------------------------------------------------------------ (O, LSE) merge
+// A block takes kRows consecutive (b, s, h) rows: phase 1 turns the two LSEs of each row
+// into weights (and writes the merged LSE), phase 2 streams the O rows as 16-byte vectors.
+// Every O element and every LSE entry is read and written by the same thread, so the
+// merged result may overwrite partial a in place.
+constexpr int kMergeRows = 64;
+constexpr int kMergeThreads = 256;
+constexpr int kMergeUnroll = 4;
+
+__device__ __forceinline__ void merge_vec_bf16(const uint4& a, const uint4& b, float wa, float wb,
+                                               uint4& o) {
+  const uint32_t* pa = &a.x;
+  const uint32_t* pb = &b.x;
+  uint32_t* po = &o.x;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float a0 = __uint_as_float(pa[e] << 16), a1 = __uint_as_float(pa[e] & 0xFFFF0000u);
+    const float b0 = __uint_as_float(pb[e] << 16), b1 = __uint_as_float(pb[e] & 0xFFFF0000u);
+    po[e] = pack_bf16x2(fmaf(wa, a0, wb * b0), fmaf(wa, a1, wb * b1));
+  }
+}
+
+__device__ __forceinline__ void merge_vec_f32(const uint4& a, const uint4& b, float wa, float wb,
+                                              uint4& o) {
+  o.x = __float_as_uint(fmaf(wa, __uint_as_float(a.x), wb * __uint_as_float(b.x)));
+  o.y = __float_as_uint(fmaf(wa, __uint_as_float(a.y), wb * __uint_as_float(b.y)));
+  o.z = __float_as_uint(fmaf(wa, __uint_as_float(a.z), wb * __uint_as_float(b.z)));
+  o.w = __float_as_uint(fmaf(wa, __uint_as_float(a.w), wb * __uint_as_float(b.w)));
+}
+
+template <bool kBf16>
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(
+    const uint4* o_a, const float* lse_a, const uint4* o_b, const float* lse_b, uint4* o,
+    float* lse, int H, int S, long long n_rows, int vpr) {
+  __shared__ float wa_s[kMergeRows], wb_s[kMergeRows];
+  for (long long r0 = (long long)blockIdx.x * kMergeRows; r0 < n_rows;
+       r0 += (long long)gridDim.x * kMergeRows) {
+    const int rows_here = int(n_rows - r0 < kMergeRows ? n_rows - r0 : kMergeRows);
+    if (threadIdx.x < rows_here) {
+      const long long row = r0 + threadIdx.x;  // (b, s, h), h fastest
+      const int h = int(row % H);
+      const long long bs = row / H;
+      const int s = int(bs % S);
+      const long long b = bs / S;
+      const long long li = (b * H + h) * S + s;
+      const float la = lse_a[li], lb = lse_b[li];
+      const float mx = fmaxf(la, lb);
+      float wa = 0.f, wb = 0.f, L = -INFINITY;
+      if (mx != -INFINITY) {
+        const float ea = expf(la - mx), eb = expf(lb - mx);
+        const float tot = ea + eb;
+        L = mx + logf(tot);
+        wa = ea / tot;
+        wb = eb / tot;
+      }
+      wa_s[threadIdx.x] = wa;
+      wb_s[threadIdx.x] = wb;
+      lse[li] = L;
+    }
+    __syncthreads();
+    const long long base = r0 * vpr;
+    const int n_vec = rows_here * vpr;
+    for (int v0 = threadIdx.x; v0 < n_vec; v0 += kMergeThreads * kMergeUnroll) {
+      uint4 a[kMergeUnroll], bb[kMergeUnroll];
+#pragma unroll
+      for (int u = 0; u < kMergeUnroll; ++u) {
+        const int v = v0 + u * kMergeThreads;
+        if (v < n_vec) {
+          a[u] = o_a[base + v];
+          bb[u] = o_b[base + v];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kMergeUnroll; ++u) {
+        const int v = v0 + u * kMergeThreads;
+        if (v < n_vec) {
+          const int rl = v / vpr;
+          uint4 r;
+          if (kBf16) merge_vec_bf16(a[u], bb[u], wa_s[rl], wb_s[rl], r);
+          else merge_vec_f32(a[u], bb[u], wa_s[rl], wb_s[rl], r);
+          o[base + v] = r;
+        }
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------ Ulysses permutes
+// Rows of Hp*D elements move as whole 16-byte-vector runs.  Head-grouped row index
+// A(g, r, s) = (g*P + r)*S_l + s; sequence-sharded row index Bq(g, r, s) = (r*S_l + s)*P + g.
+// seq2head: dst[A] = src[Bq]; head2seq: dst[Bq] = src[A].  Threads walk dst rows in order
+// (coalesced stores); each warp moves kPermUnroll (row, 32-vector chunk) items at a time.
+constexpr int kPermThreads = 256;
+constexpr int kPermUnroll = 4;
+
+template <bool kToHead>
+__global__ void __launch_bounds__(kPermThreads) permute_kernel(const uint4* __restrict__ src,
+                                                                uint4* __restrict__ dst, int P,
+                                                                int S_l, int run_vec, int chunks,
+                                                                long long n_items) {
+  const int lane = threadIdx.x & 31;
+  const long long warp = ((long long)blockIdx.x * kPermThreads + threadIdx.x) >> 5;
+  const long long n_warps = ((long long)gridDim.x * kPermThreads) >> 5;
+  for (long long it0 = warp * kPermUnroll; it0 < n_items; it0 += n_warps * kPermUnroll) {
+    uint4 buf[kPermUnroll];
+    long long dst_off[kPermUnroll];
+    bool live[kPermUnroll];
+#pragma unroll
+    for (int u = 0; u < kPermUnroll; ++u) {
+      const long long it = it0 + u;
+      const long long n = it / chunks;  // dst row
+      const int v = int(it - n * chunks) * 32 + lane;
+      live[u] = it < n_items && v < run_vec;
+      long long src_row = 0;
+      if (kToHead) {  // n = A(g, r, s)
+        const int s = int(n % S_l);
+        const long long gr = n / S_l;
+        const int r = int(gr % P);
+        const int g = int(gr / P);
+        src_row = ((long long)r * S_l + s) * P + g;
+      } else {  // n = Bq(g, r, s)
+        const int g = int(n % P);
+        const long long rs = n / P;
+        const int s = int(rs % S_l);
+        const int r = int(rs / S_l);
+        src_row = ((long long)g * P + r) * S_l + s;
+      }
+      dst_off[u] = n * run_vec + v;
+      if (live[u]) buf[u] = src[src_row * run_vec + v];
+    }
+#pragma unroll
+    for (int u = 0; u < kPermUnroll; ++u)
+      if (live[u]) dst[dst_off[u]] = buf[u];
+  }
+}
+
+// ------------------------------------------------------------------ bounded-wait self-test
+__global__ void wait_timeout_selftest_kernel(int* err, long long limit) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_sh;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_sh = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // nothing ever arrives on `bar`: the wait must run out and record the timeout
+  mbar_wait(smem_u32(&bar), 0, &abort_sh, err, limit);
+  __syncthreads();
+}
+
+long long grid_for(long long work_items, int threads, int waves_per_sm) {
+  const long long per_block = threads;
+  long long blocks = (work_items + per_block - 1) / per_block;
+  const long long cap = (long long)sm_count() * waves_per_sm;
+  if (blocks > cap) blocks = cap;
+  return blocks < 1 ? 1 : blocks;
+}
+
+}  // namespace
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+cudaError_t launch_attn_fwd_f32(const float* q, const float* k, const float* v, void* out,
+                                float* lse, int B, int H, int Sq, int Skv, int D, float scale,
+                                bool out_bf16, cudaStream_t stream) {
+  const long long rows = (long long)B * H * Sq;
+  const int warps = 8;
+  const long long blocks = (rows + warps - 1) / warps;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  const int T = (D + 31) / 32;
+#define CPATTN_F32_CASE(TT)                                                                   \
+  case TT:                                                                                    \
+    attn_f32_kernel<TT><<<unsigned(blocks), warps * 32, 0, stream>>>(q, k, v, out, lse, B, H, \
+                                                                     Sq, Skv, D, scale,       \
+                                                                     out_bf16);               \
+    break;
+  switch (T) {
+    CPATTN_F32_CASE(1)
+    CPATTN_F32_CASE(2)
+    CPATTN_F32_CASE(3)
+    CPATTN_F32_CASE(4)
+    CPATTN_F32_CASE(5)
+    CPATTN_F32_CASE(6)
+    CPATTN_F32_CASE(7)
+    CPATTN_F32_CASE(8)
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef CPATTN_F32_CASE
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fill_empty(void* out, size_t out_bytes, float* lse, size_t n_lse,
+                              cudaStream_t stream) {
+  const size_t n_vec = out_bytes / 16;
+  const long long work = (long long)(n_vec > n_lse ? n_vec : n_lse);
+  fill_empty_kernel<<<unsigned(grid_for(work, 256, 8)), 256, 0, stream>>>(
+      static_cast<uint4*>(out), n_vec, lse, n_lse);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
+                         void* o, float* lse, int B, int H, int S, int D, int elem_bytes,
+                         cudaStream_t stream) {
+  const long long n_rows = (long long)B * S * H;
+  const int vpr = D * elem_bytes / 16;
+  const long long blocks_needed = (n_rows + kMergeRows - 1) / kMergeRows;
+  long long cap = (long long)sm_count() * 8;  // 8 resident 256-thread blocks per SM
+  const long long blocks = blocks_needed < cap ? blocks_needed : cap;
+  if (elem_bytes == 2)
+    merge_kernel<true><<<unsigned(blocks), kMergeThreads, 0, stream>>>(
+        static_cast<const uint4*>(o_a), lse_a, static_cast<const uint4*>(o_b), lse_b,
+        static_cast<uint4*>(o), lse, H, S, n_rows, vpr);
+  else
+    merge_kernel<false><<<unsigned(blocks), kMergeThreads, 0, stream>>>(
+        static_cast<const uint4*>(o_a), lse_a, static_cast<const uint4*>(o_b), lse_b,
+        static_cast<uint4*>(o), lse, H, S, n_rows, vpr);
+  return cudaGetLastError();
+}
+
+static cudaError_t launch_permute(bool to_head, const void* src, void* dst, int P, int S_local,
+                                  long long run_vec, cudaStream_t stream) {
+  const long long n_rows = (long long)P * P * S_local;
+  const int chunks = int((run_vec + 31) / 32);
+  const long long n_items = n_rows * chunks;
+  const long long warps_needed = (n_items + kPermUnroll - 1) / kPermUnroll;
+  const long long blocks_needed = (warps_needed * 32 + kPermThreads - 1) / kPermThreads;
+  const long long cap = (long long)sm_count() * 8;
+  const long long blocks = blocks_needed < cap ? blocks_needed : cap;
+  if (to_head)
+    permute_kernel<true><<<unsigned(blocks), kPermThreads, 0, stream>>>(
+        static_cast<const uint4*>(src), static_cast<uint4*>(dst), P, S_local, int(run_vec), chunks,
+        n_items);
+  else
+    permute_kernel<false><<<unsigned(blocks), kPermThreads, 0, stream>>>(
+        static_cast<const uint4*>(src), static_cast<uint4*>(dst), P, S_local, int(run_vec), chunks,
+        n_items);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_seq2head(const void* src, void* dst, int P, int S_local, long long run_vec,
+                            cudaStream_t stream) {
+  return launch_permute(true, src, dst, P, S_local, run_vec, stream);
+}
+
+cudaError_t launch_head2seq(const void* src, void* dst, int P, int S_local, long long run_vec,
+                            cudaStream_t stream) {
+  return launch_permute(false, src, dst, P, S_local, run_vec, stream);
+}
+
+cudaError_t launch_wait_timeout_selftest(int* err, long long limit, cudaStream_t stream) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(err, limit);
+  return cudaGetLastError();
+}
+
+}  // namespace cpattn

@@ -1,0 +1,80 @@
+"""The two per-rank compositions of the hot path, built from the C-ABI calls.
+
+* Ring Attention step (环形注意力 section of the TensorRT multi-device blog, Fig. 3): a
+  rank keeps its Q slice and folds the partial (O, LSE) of each arriving K/V chunk into a
+  running result with the exact online-softmax merge.
+* DeepSpeed Ulysses (Fig. 4): all-to-all from sequence shards to head groups, attention
+  over the full sequence per head group, all-to-all back; here the all-to-alls are local
+  permutes over P virtual ranks on one GPU.
+
+Buffers come from PyTorch (device memory only); every step is a libcpattn kernel.
+"""
+
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import _binding as B
+
+
+def ring_attention(q, k_chunks, v_chunks, scale=None, acc_dtype=None, stream=None):
+    """One rank's ring step over K/V chunks in ring order.
+
+    q: [B][Sq][H][D]; each chunk [B][S_c][H][D].  The running (O, LSE) is kept in
+    ``acc_dtype`` (default: q's dtype); chunk partials are produced in the same dtype and
+    merged in place.  Returns ``(O, LSE)``.
+    """
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[3])
+    acc_dtype = acc_dtype or q.dtype
+    Bn, Sq, H, D = q.shape
+    acc_o = torch.empty((Bn, Sq, H, D), dtype=acc_dtype, device=q.device)
+    acc_l = torch.empty((Bn, H, Sq), dtype=torch.float32, device=q.device)
+    tmp_o = torch.empty_like(acc_o)
+    tmp_l = torch.empty_like(acc_l)
+    for c, (kc, vc) in enumerate(zip(k_chunks, v_chunks)):
+        if c == 0:
+            B.fwd(q, kc, vc, out=acc_o, lse=acc_l, scale=scale, stream=stream)
+        else:
+            B.fwd(q, kc, vc, out=tmp_o, lse=tmp_l, scale=scale, stream=stream)
+            B.merge(acc_o, acc_l, tmp_o, tmp_l, out=acc_o, lse=acc_l, stream=stream)
+    return acc_o, acc_l
+
+
+class UlyssesPlan:
+    """Preallocated buffers for the Ulysses path over P virtual ranks.
+
+    Shards are [P][S_l][H][D]; head-grouped buffers [P][P*S_l][H/P][D].
+    """
+
+    def __init__(self, P, S_local, H, D, dtype=torch.bfloat16, device="cuda"):
+        if H % P:
+            raise ValueError("H must be divisible by P")
+        self.P, self.S_local, self.H, self.D = P, S_local, H, D
+        grouped = (P, P * S_local, H // P, D)
+        self.qh = torch.empty(grouped, dtype=dtype, device=device)
+        self.kh = torch.empty(grouped, dtype=dtype, device=device)
+        self.vh = torch.empty(grouped, dtype=dtype, device=device)
+        self.oh = torch.empty(grouped, dtype=dtype, device=device)
+        self.lse = torch.empty((P, H // P, P * S_local), dtype=torch.float32, device=device)
+        self.out = torch.empty((P, S_local, H, D), dtype=dtype, device=device)
+
+    def run(self, q_shards, k_shards, v_shards, scale=None, stream=None):
+        P = self.P
+        B.seq2head(q_shards, P, out=self.qh, stream=stream)
+        B.seq2head(k_shards, P, out=self.kh, stream=stream)
+        B.seq2head(v_shards, P, out=self.vh, stream=stream)
+        B.fwd(self.qh, self.kh, self.vh, out=self.oh, lse=self.lse, scale=scale, stream=stream)
+        B.head2seq(self.oh, P, out=self.out, stream=stream)
+        return self.out, self.lse
+
+
+def ulysses_attention(q_shards, k_shards, v_shards, P, scale=None, stream=None):
+    """seq2head x3 -> attention per head group -> head2seq.  Returns
+    ``(O [P][S_l][H][D], LSE [P][H/P][P*S_l])``."""
+    P_, S_l, H, D = q_shards.shape
+    plan = UlyssesPlan(P, S_l, H, D, dtype=q_shards.dtype, device=q_shards.device)
+    out, lse = plan.run(q_shards, k_shards, v_shards, scale=scale, stream=stream)
+    return out, lse

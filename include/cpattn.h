@@ -1,0 +1,160 @@
+/*
+ * cpattn.h -- C ABI of the per-rank context-parallel attention hot path (B200, sm_100a).
+ *
+ * The operations come from the context-parallel attention strategies described in
+ * "Scaling AI Inference Across Multiple GPUs Using NVIDIA TensorRT with Multi-Device
+ * Inference Support" (NVIDIA developer blog): AllGather KV (Fig. 2), 环形注意力 /
+ * Ring Attention with online softmax (Fig. 3) and DeepSpeed Ulysses (Fig. 4).  The
+ * pages print no interface for this compute; the calls below are this library's own.
+ *
+ * Layout of every activation tensor (reading of the (seq, batch, heads, dim) reshape in
+ * the attention_mdtrt guide "TensorRT 多设备注意力推理实战", section 模型的核心结构):
+ *   Q, K, V, O : [B][S][H][D] row-major (token-major, heads interleaved, D contiguous)
+ *   LSE        : [B][H][Sq]  float32, natural log of the sum of exp of the scaled logits
+ *
+ * Conventions shared by every call
+ *   - Ownership: the caller allocates and owns every buffer (device memory unless a
+ *     call says otherwise).  The library allocates nothing per call; it keeps one
+ *     device error word per device for bounded-wait timeouts.
+ *   - Asynchrony: work is enqueued on `stream` (NULL = legacy default stream) and the
+ *     call returns without waiting.  Argument errors are detected on the host, before
+ *     anything is launched, and nothing is written then.
+ *   - Return value: a cpattn_status.  CPATTN_ERR_CUDA means a launch failed; the CUDA
+ *     error is left for the caller's next CUDA call to report as well.
+ *   - Tensor pointers (Q, K, V, O, permute buffers) must be 16-byte aligned and LSE
+ *     pointers 4-byte aligned (CPATTN_ERR_ALIGN otherwise).
+ *   - Every argument is checked before the first CUDA call, so argument errors are
+ *     reported the same way with or without a GPU.
+ */
+#ifndef CPATTN_H
+#define CPATTN_H
+
+#if defined(__GNUC__)
+#define CPATTN_API __attribute__((visibility("default")))
+#else
+#define CPATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream; declared here so this header needs no CUDA
+ * include. */
+typedef struct CUstream_st* cpattn_stream_t;
+
+typedef enum {
+  CPATTN_BF16 = 0, /* bfloat16, round-to-nearest-even on output */
+  CPATTN_F32 = 1   /* IEEE float32 */
+} cpattn_dtype;
+
+typedef enum {
+  CPATTN_OK = 0,
+  CPATTN_ERR_NULL = 1,        /* a required pointer is NULL */
+  CPATTN_ERR_SHAPE = 2,       /* a size is out of range or inconsistent */
+  CPATTN_ERR_ALIGN = 3,       /* a pointer is not suitably aligned */
+  CPATTN_ERR_UNSUPPORTED = 4, /* valid request this build has no kernel for */
+  CPATTN_ERR_CUDA = 5,        /* a CUDA runtime/driver call or launch failed */
+  CPATTN_ERR_DEVICE_TIMEOUT = 6 /* a kernel's bounded wait ran out (device error word) */
+} cpattn_status;
+
+/*
+ * cpattn_fwd -- non-causal scaled dot-product attention with its log-sum-exp.
+ *
+ * Defines (AllGather KV and Ring Attention sections, Figs. 2-3; the QK^T -> Softmax ->
+ * Attn*V core of the attention_mdtrt guide):
+ *   s[b,h,i,j] = scale * sum_d q[b,i,h,d] * k[b,j,h,d]
+ *   lse[b,h,i] = ln sum_j exp(s[b,h,i,j])
+ *   out[b,i,h,:] = sum_j exp(s[b,h,i,j] - lse[b,h,i]) * v[b,j,h,:]
+ * No mask.  With Sq != Skv this is one rank's AllGather-KV attention or one Ring
+ * Attention chunk; the (out, lse) pair is what cpattn_merge folds.
+ *
+ * q   : [B][Sq][H][D]  in_dtype        k, v : [B][Skv][H][D] in_dtype
+ * out : [B][Sq][H][D]  out_dtype       lse  : [B][H][Sq] float32, or NULL to skip it
+ * B, H, Sq >= 1; Skv >= 0 (Skv = 0 gives out = 0, lse = -inf; k and v may be NULL).
+ * scale must be finite and > 0 (the usual 1/sqrt(D)); the row maximum the kernel
+ * subtracts for stability is taken on the unscaled logits.
+ * in_dtype CPATTN_BF16: tensor-core kernel (tcgen05, TMEM accumulators, TMA-fed),
+ *   D must be 64 or 128, fp32 accumulation and softmax; out_dtype BF16 (production)
+ *   or F32 (same kernel, fp32 epilogue, for verification).
+ * in_dtype CPATTN_F32: fp32 CUDA-core kernel, 1 <= D <= 256, out_dtype F32 or BF16.
+ * Errors: CPATTN_ERR_NULL, _SHAPE, _ALIGN, _UNSUPPORTED (dtype/D combination),
+ *   _CUDA.  A bounded wait that runs out inside the kernel is reported by
+ *   cpattn_device_error(), not by this call (it returns before the kernel runs).
+ */
+CPATTN_API int cpattn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+               int B, int H, int Sq, int Skv, int D, float scale,
+               int in_dtype, int out_dtype, cpattn_stream_t stream);
+
+/*
+ * cpattn_merge -- exact merge of two partial attention results over disjoint key sets
+ * (the Ring Attention step: each rank folds each arriving K/V chunk's partial into its
+ * running result with the online softmax, Fig. 3):
+ *   L = max(La, Lb) + ln(exp(La - max) + exp(Lb - max))
+ *   O = exp(La - L) * Oa + exp(Lb - L) * Ob
+ * Two empty partials (La = Lb = -inf) give O = 0, L = -inf (never NaN).
+ *
+ * o_a, o_b, o : [B][S][H][D] in `dtype` (BF16 or F32); math in fp32.
+ * lse_a, lse_b, lse : [B][H][S] float32.
+ * o may alias o_a and lse may alias lse_a (in-place accumulate); no other overlap.
+ * D must be a multiple of 8 (BF16) or 4 (F32) so rows move as 16-byte vectors.
+ * Errors: CPATTN_ERR_NULL, _SHAPE, _ALIGN, _UNSUPPORTED (dtype), _CUDA.
+ */
+CPATTN_API int cpattn_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
+                 void* o, float* lse, int B, int H, int S, int D, int dtype,
+                 cpattn_stream_t stream);
+
+/*
+ * cpattn_seq2head -- the DeepSpeed Ulysses first all-to-all (Fig. 4), run locally over
+ * P virtual ranks: every rank's sequence shard becomes a full-sequence tensor of one
+ * contiguous head group.  With Hp = H / P:
+ *   dst[g][r*S_local + s][j][d] = src[r][s][g*Hp + j][d]
+ * src : [P][S_local][H][D], dst : [P][P*S_local][Hp][D]; elements are copied as raw
+ * `elem_bytes`-byte words (2 or 4), so the result is bit-exact.  dst is itself a
+ * BSHD tensor with B = P, H = Hp, S = P*S_local, ready for cpattn_fwd.
+ * Requires H % P == 0, Hp*D*elem_bytes a multiple of 16, src and dst not overlapping.
+ * Errors: CPATTN_ERR_NULL, _SHAPE, _ALIGN, _CUDA.
+ */
+CPATTN_API int cpattn_seq2head(const void* src, void* dst, int P, int S_local, int H, int D,
+                    int elem_bytes, cpattn_stream_t stream);
+
+/*
+ * cpattn_head2seq -- the Ulysses second all-to-all (Fig. 4), exact inverse of
+ * cpattn_seq2head:
+ *   dst[r][s][g*Hp + j][d] = src[g][r*S_local + s][j][d]
+ * src : [P][P*S_local][Hp][D] with Hp = H / P, dst : [P][S_local][H][D].
+ * Same requirements and errors as cpattn_seq2head.
+ */
+CPATTN_API int cpattn_head2seq(const void* src, void* dst, int P, int S_local, int H, int D,
+                    int elem_bytes, cpattn_stream_t stream);
+
+/* Human-readable name of a cpattn_status value (static string, never NULL). */
+CPATTN_API const char* cpattn_status_str(int status);
+
+/*
+ * cpattn_device_error -- synchronizes the current device, then reads and clears its
+ * device error word.  Returns CPATTN_OK, or CPATTN_ERR_DEVICE_TIMEOUT if a kernel's
+ * bounded wait (mbarrier / pipeline) ran out since the last call, or CPATTN_ERR_CUDA
+ * if the synchronization itself failed.
+ */
+CPATTN_API int cpattn_device_error(void);
+
+/*
+ * cpattn_selftest_wait_timeout -- launches one CTA that waits on a pipeline barrier
+ * nothing will ever complete, through the same bounded-wait routine the attention
+ * kernel uses, with a limit of `limit_cycles` SM clock cycles (1 .. 2^31).  The wait
+ * runs out, the kernel records the timeout in the device error word and returns, so
+ * cpattn_device_error() must then report CPATTN_ERR_DEVICE_TIMEOUT.  Used by tests to
+ * show a stalled pipeline ends in an error status instead of a hang.
+ * Errors: CPATTN_ERR_SHAPE (limit out of range), _CUDA.
+ */
+CPATTN_API int cpattn_selftest_wait_timeout(long long limit_cycles, cpattn_stream_t stream);
+
+/* ABI version: (major << 16) | minor. */
+CPATTN_API int cpattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CPATTN_H */

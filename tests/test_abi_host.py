@@ -1,0 +1,117 @@
+"""Host-only checks of the C ABI (no GPU): the library builds and loads, exports every
+symbol include/cpattn.h declares, and rejects bad arguments before any CUDA call."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from context_long_sequence_non_b200 import _binding as B
+from context_long_sequence_non_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build_mod.build()
+    return B.lib()
+
+
+def _declared():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            with open(os.path.join(ROOT, "include", fn)) as f:
+                names += re.findall(r"CPATTN_API\s+[\w\s\*]+?\b(cpattn_\w+)\s*\(", f.read())
+    return names
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert {"cpattn_fwd", "cpattn_merge", "cpattn_seq2head", "cpattn_head2seq",
+            "cpattn_status_str", "cpattn_device_error"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_version_and_status_strings(L):
+    assert B.version() >> 16 == 1
+    for s in range(7):
+        assert B.status_str(s).startswith("CPATTN")
+    assert "unknown" in B.status_str(99)
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails validation
+
+
+def fwd(L, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B_=1, H=2, Sq=8, Skv=8, D=128, scale=0.1,
+        din=0, dout=0):
+    vp = ctypes.c_void_p
+    return L.cpattn_fwd(vp(q) if q else None, vp(k) if k else None, vp(v) if v else None,
+                        vp(o) if o else None, vp(lse) if lse else None, B_, H, Sq, Skv, D,
+                        scale, din, dout, None)
+
+
+def test_fwd_argument_errors(L):
+    assert fwd(L, Sq=0) == B.ERR_SHAPE
+    assert fwd(L, Skv=-1) == B.ERR_SHAPE
+    assert fwd(L, D=0) == B.ERR_SHAPE
+    assert fwd(L, scale=0.0) == B.ERR_SHAPE
+    assert fwd(L, scale=-1.0) == B.ERR_SHAPE
+    assert fwd(L, scale=float("inf")) == B.ERR_SHAPE
+    assert fwd(L, din=7) == B.ERR_UNSUPPORTED
+    assert fwd(L, q=0) == B.ERR_NULL
+    assert fwd(L, o=0) == B.ERR_NULL
+    assert fwd(L, k=0) == B.ERR_NULL
+    assert fwd(L, q=FAKE + 8) == B.ERR_ALIGN
+    assert fwd(L, v=FAKE + 2) == B.ERR_ALIGN
+    assert fwd(L, lse=FAKE + 2) == B.ERR_ALIGN
+    assert fwd(L, D=96) == B.ERR_UNSUPPORTED  # bf16 tensor-core kernel: D in {64, 128}
+    assert fwd(L, D=264, din=1, dout=1) == B.ERR_UNSUPPORTED  # fp32 kernel: D <= 256
+    assert fwd(L, B_=70000) == B.ERR_SHAPE
+
+
+def test_merge_argument_errors(L):
+    vp = ctypes.c_void_p
+    base = [vp(FAKE), vp(FAKE + 0x100000), vp(FAKE + 0x200000), vp(FAKE + 0x300000),
+            vp(FAKE + 0x400000), vp(FAKE + 0x500000)]
+
+    def merge(ptrs=base, B_=1, H=2, S=4, D=128, dt=0):
+        return L.cpattn_merge(*ptrs, B_, H, S, D, dt, None)
+
+    assert merge(S=0) == B.ERR_SHAPE
+    assert merge(D=12) == B.ERR_SHAPE  # 24 bytes: not a whole number of 16-byte vectors
+    assert merge(dt=5) == B.ERR_UNSUPPORTED
+    assert merge(ptrs=[None] + base[1:]) == B.ERR_NULL
+    assert merge(ptrs=base[:4] + [vp(FAKE + 0x400008)] + base[5:]) == B.ERR_ALIGN
+    # o overlapping o_b (not the allowed o == o_a in-place case)
+    assert merge(ptrs=base[:4] + [vp(FAKE + 0x200000 + 16)] + base[5:]) == B.ERR_SHAPE
+
+
+def test_permute_argument_errors(L):
+    vp = ctypes.c_void_p
+    s, d = vp(FAKE), vp(FAKE + 0x1000000)
+    for fn in (L.cpattn_seq2head, L.cpattn_head2seq):
+        assert fn(s, d, 3, 4, 16, 128, 2, None) == B.ERR_SHAPE  # H % P != 0
+        assert fn(s, d, 2, 4, 16, 128, 3, None) == B.ERR_SHAPE  # elem_bytes
+        assert fn(s, d, 16, 4, 16, 4, 2, None) == B.ERR_SHAPE   # 8-byte runs
+        assert fn(None, d, 2, 4, 16, 128, 2, None) == B.ERR_NULL
+        assert fn(vp(FAKE + 4), d, 2, 4, 16, 128, 2, None) == B.ERR_ALIGN
+        assert fn(s, vp(FAKE + 64), 2, 4, 16, 128, 2, None) == B.ERR_SHAPE  # overlap
+
+
+def test_selftest_limit_checked(L):
+    assert L.cpattn_selftest_wait_timeout(0, None) == B.ERR_SHAPE
+    assert L.cpattn_selftest_wait_timeout((1 << 31) + 1, None) == B.ERR_SHAPE
+
+
+def test_product_path_has_no_oracle_or_fallback():
+    pkg = os.path.join(ROOT, "context_long_sequence_non_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                with open(os.path.join(dirpath, fn)) as f:
+                    src = f.read()
+                assert "import oracle" not in src and "from oracle" not in src, fn

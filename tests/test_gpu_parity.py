@@ -1,0 +1,330 @@
+"""GPU parity: every kernel of the path, called through the C ABI (libcpattn.so via the
+ctypes binding), against the fp64 CPU oracle on the same seeded inputs.
+
+Small cases compare every element; the five workloads run at full size and compare
+sampled rows (each sampled row exact in the oracle) plus properties that hold at any size.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import context_long_sequence_non_b200 as cp
+from context_long_sequence_non_b200 import build as build_mod
+from context_long_sequence_non_b200 import workloads as W
+from context_long_sequence_non_b200.paths import UlyssesPlan
+from oracle import ref
+from parity import check_lse, check_o, half_ulp_bf16, rel_l2, to64
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    build_mod.build()
+    cp.lib()
+    yield
+    assert cp.device_error() == 0, "a kernel's bounded wait ran out during this module"
+
+
+def bits(t):
+    return t.view(torch.int16 if t.element_size() == 2 else torch.int32)
+
+
+# ----------------------------------------------------------------------------- permutes
+
+
+@pytest.mark.parametrize("P,S_l,H,D,dt", [(2, 3, 4, 8, torch.bfloat16), (4, 5, 8, 16, torch.float32),
+                                          (1, 7, 2, 64, torch.bfloat16), (8, 33, 16, 128, torch.bfloat16),
+                                          (3, 10, 6, 8, torch.bfloat16), (2, 1, 2, 8, torch.float32)])
+def test_permutes_bit_exact(P, S_l, H, D, dt):
+    g = torch.Generator().manual_seed(P * 1000 + S_l)
+    ib = torch.int16 if dt == torch.bfloat16 else torch.int32
+    lim = 1 << (15 if ib == torch.int16 else 31)
+    src_bits = torch.randint(-lim, lim, (P, S_l, H, D), generator=g, dtype=torch.int64).to(ib)
+    src = src_bits.view(dt).to(DEV)
+    dst = cp.seq2head(src, P)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(bits(dst).cpu().numpy(), ref.seq2head(src_bits.numpy(), P))
+    back = cp.head2seq(dst, P)
+    torch.cuda.synchronize()
+    assert torch.equal(bits(back).cpu(), src_bits)
+
+
+def test_permutes_ulysses_full_size_bit_exact():
+    P, S_l, H, D = 8, W.ULYSSES_LOCAL_TOKENS, W.ULYSSES_HEADS, 128
+    g = torch.Generator().manual_seed(77)
+    src_bits = torch.randint(-32768, 32768, (P, S_l, H, D), generator=g, dtype=torch.int32).to(torch.int16)
+    src = src_bits.view(torch.bfloat16).to(DEV)
+    dst = cp.seq2head(src, P)
+    back = cp.head2seq(dst, P)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(bits(dst).cpu().numpy(), ref.seq2head(src_bits.numpy(), P))
+    assert torch.equal(bits(back).cpu(), src_bits)
+
+
+# ----------------------------------------------------------------------------- merge
+
+
+def _rand_partials(seed, Bn, S, H, D, dt, empty_frac=0.0):
+    g = torch.Generator().manual_seed(seed)
+    oa = torch.randn(Bn, S, H, D, generator=g).to(dt)
+    ob = torch.randn(Bn, S, H, D, generator=g).to(dt)
+    la = torch.randn(Bn, H, S, generator=g) * 5
+    lb = torch.randn(Bn, H, S, generator=g) * 5
+    if empty_frac:
+        ma = torch.rand(Bn, H, S, generator=g) < empty_frac
+        mb = torch.rand(Bn, H, S, generator=g) < empty_frac
+        la[ma] = -math.inf
+        lb[mb] = -math.inf
+    return oa, la, ob, lb
+
+
+def _check_merge(o, l, oa, la, ob, lb, dt, what):
+    o_ref, l_ref = ref.merge(oa, la, ob, lb)
+    scale = np.abs(to64(oa)) + np.abs(to64(ob))
+    err = np.abs(to64(o) - o_ref)
+    bound = 1e-6 * scale + 1e-7 + (half_ulp_bf16(o_ref) if dt == torch.bfloat16 else 0.0)
+    assert (err <= bound).all(), f"{what}: merge O err {err.max():.3e}"
+    l64 = to64(l)
+    assert (np.isneginf(l64) == np.isneginf(l_ref)).all()
+    fin = ~np.isneginf(l_ref)
+    assert (np.abs(l64[fin] - l_ref[fin]) <= 1e-5 * np.maximum(1, np.abs(l_ref[fin]))).all()
+    assert not np.isnan(to64(o)).any()
+
+
+@pytest.mark.parametrize("Bn,S,H,D,dt,empty", [(2, 37, 3, 64, torch.bfloat16, 0.0),
+                                              (1, 5520, 16, 128, torch.bfloat16, 0.0),
+                                              (2, 19, 2, 32, torch.float32, 0.0),
+                                              (1, 300, 4, 128, torch.bfloat16, 0.3),
+                                              (1, 64, 2, 8, torch.float32, 0.5)])
+def test_merge_matches_oracle(Bn, S, H, D, dt, empty):
+    oa, la, ob, lb = _rand_partials(S + D, Bn, S, H, D, dt, empty)
+    o, l = cp.merge(oa.to(DEV), la.to(DEV), ob.to(DEV), lb.to(DEV))
+    torch.cuda.synchronize()
+    _check_merge(o, l, oa, la, ob, lb, dt, "out-of-place")
+    # in place: the running partial is overwritten (the ring accumulator)
+    a_o, a_l = oa.to(DEV), la.to(DEV)
+    cp.merge(a_o, a_l, ob.to(DEV), lb.to(DEV), out=a_o, lse=a_l)
+    torch.cuda.synchronize()
+    _check_merge(a_o, a_l, oa, la, ob, lb, dt, "in-place")
+
+
+# ----------------------------------------------------------------------------- fp32 attention
+
+
+def test_f32_config1_full_and_chunked():
+    w = W.WORKLOADS[1]
+    x = W.make_inputs(w)
+    q, k, v = (x[n].to(DEV) for n in ("q", "k", "v"))
+    o_ref, l_ref = ref.attention(x["q"], x["k"], x["v"], w.softmax_scale)
+    o, l = cp.fwd(q, k, v, scale=w.softmax_scale)
+    torch.cuda.synchronize()
+    check_o(o, o_ref, "f32", "config 1 single pass")
+    check_lse(l, l_ref, "config 1", tol=1e-5)
+    # 2 chunks of 128 keys merged == unchunked
+    c0 = x["chunks"][0]
+    oa, la = cp.fwd(q, k[:, :c0].contiguous(), v[:, :c0].contiguous(), scale=w.softmax_scale)
+    ob, lb = cp.fwd(q, k[:, c0:].contiguous(), v[:, c0:].contiguous(), scale=w.softmax_scale)
+    om, lm = cp.merge(oa, la, ob, lb)
+    torch.cuda.synchronize()
+    check_o(om, o_ref, "f32", "config 1 chunked + merge")
+    check_lse(lm, l_ref, "config 1 chunked", tol=1e-5)
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 1, 1, 1), (2, 3, 17, 29, 40), (1, 2, 5, 300, 256)])
+def test_f32_odd_shapes(shape):
+    Bn, H, Sq, Skv, D = shape
+    q, k, v = W.random_case(sum(shape), Bn, H, Sq, Skv, D, dtype="f32")
+    o, l = cp.fwd(q.to(DEV), k.to(DEV), v.to(DEV), scale=0.3)
+    torch.cuda.synchronize()
+    o_ref, l_ref = ref.attention(q, k, v, 0.3)
+    check_o(o, o_ref, "f32", str(shape))
+    check_lse(l, l_ref, str(shape), tol=1e-5)
+
+
+# ----------------------------------------------------------------------------- bf16 tensor-core attention
+
+SHAPES = [(1, 1, 1, 1, 128), (1, 2, 17, 33, 128), (2, 3, 128, 128, 128), (1, 2, 129, 257, 128),
+          (1, 1, 300, 1000, 128), (2, 2, 255, 129, 64), (1, 4, 1000, 77, 64), (1, 1, 513, 1, 128),
+          (1, 1, 3, 3000, 128), (3, 1, 256, 384, 128), (1, 2, 640, 640, 64)]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_bf16_shapes_match_oracle(shape):
+    Bn, H, Sq, Skv, D = shape
+    q, k, v = W.random_case(hash(shape) % 10000, Bn, H, Sq, Skv, D)
+    scale = 1.0 / math.sqrt(D)
+    o_ref, l_ref = ref.attention(q, k, v, scale)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    o32, l32 = cp.fwd(qd, kd, vd, scale=scale, out_dtype=torch.float32)
+    o16, l16 = cp.fwd(qd, kd, vd, scale=scale)
+    torch.cuda.synchronize()
+    check_o(o32, o_ref, "bf16_in", f"{shape} fp32 epilogue")
+    check_o(o16, o_ref, "bf16_out", f"{shape} bf16 out")
+    check_lse(l32, l_ref, str(shape))
+    assert torch.equal(l16, l32)
+    assert rel_l2(o32, o_ref) < 1e-2
+
+
+def test_bf16_large_logits_stable():
+    q, k, v = W.random_case(5, 1, 2, 300, 700, 128, sigma_qk=3.0)
+    scale = 1.0 / math.sqrt(128)
+    o_ref, l_ref = ref.attention(q, k, v, scale)
+    o, l = cp.fwd(q.to(DEV), k.to(DEV), v.to(DEV), scale=scale, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    check_o(o, o_ref, "bf16_in", "sigma 3")
+    check_lse(l, l_ref, "sigma 3")
+
+
+def test_empty_key_set():
+    q = torch.randn(1, 5, 2, 128).to(torch.bfloat16).to(DEV)
+    e = torch.empty(1, 0, 2, 128, dtype=torch.bfloat16, device=DEV)
+    o, l = cp.fwd(q, e, e)
+    torch.cuda.synchronize()
+    assert torch.all(o == 0) and torch.all(torch.isneginf(l))
+
+
+def test_guard_bands_untouched():
+    Bn, H, Sq, Skv, D = 1, 2, 200, 300, 128
+    q, k, v = (t.to(DEV) for t in W.random_case(9, Bn, H, Sq, Skv, D))
+    G, n_o, n_l = 4096, Bn * Sq * H * D, Bn * H * Sq
+    o_buf = torch.full((n_o + 2 * G,), 7.0, dtype=torch.bfloat16, device=DEV)
+    l_buf = torch.full((n_l + 2 * G,), 7.0, dtype=torch.float32, device=DEV)
+    o = o_buf[G:G + n_o].view(Bn, Sq, H, D)
+    l = l_buf[G:G + n_l].view(Bn, H, Sq)
+    cp.fwd(q, k, v, out=o, lse=l)
+    torch.cuda.synchronize()
+    for buf, n in ((o_buf, n_o), (l_buf, n_l)):
+        assert torch.all(buf[:G] == 7.0) and torch.all(buf[G + n:] == 7.0)
+    assert torch.isfinite(l).all() and torch.isfinite(o.float()).all()
+
+
+def test_invariants_on_gpu():
+    Bn, H, Sq, Skv, D = 1, 2, 130, 517, 128
+    q, k, v = W.random_case(11, Bn, H, Sq, Skv, D)
+    scale = 1.0 / math.sqrt(D)
+    kd, vd = k.to(DEV), v.to(DEV)
+    # Q = 0: every row is the column mean of V, LSE = ln Skv
+    o0, l0 = cp.fwd(torch.zeros_like(q).to(DEV), kd, vd, scale=scale, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    mean_v = to64(v).mean(axis=1, keepdims=True)
+    check_o(o0, np.broadcast_to(mean_v, o0.shape), "bf16_in", "Q=0")
+    check_lse(l0, np.full(l0.shape, math.log(Skv)), "Q=0")
+    # joint permutation of K/V rows leaves O and LSE unchanged
+    perm = torch.randperm(Skv, generator=torch.Generator().manual_seed(3))
+    qd = q.to(DEV)
+    o1, l1 = cp.fwd(qd, kd, vd, scale=scale, out_dtype=torch.float32)
+    o2, l2 = cp.fwd(qd, kd[:, perm].contiguous(), vd[:, perm].contiguous(), scale=scale,
+                    out_dtype=torch.float32)
+    # duplicated K/V: O unchanged, LSE + ln 2
+    o3, l3 = cp.fwd(qd, torch.cat([kd, kd], 1), torch.cat([vd, vd], 1), scale=scale,
+                    out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert (o1 - o2).abs().max().item() < 2e-3 and (l1 - l2).abs().max().item() < 1e-4
+    assert (o1 - o3).abs().max().item() < 2e-3
+    assert ((l3 - l1) - math.log(2)).abs().max().item() < 1e-4
+
+
+# ----------------------------------------------------------------------------- the five workloads
+
+
+def _sampled(q, k, v, scale, o, l, rows, kind, what):
+    o_ref, l_ref = ref.attention_rows(q, k, v, scale, rows)
+    o_rows = torch.stack([o[b, i, h] for (b, h, i) in rows])
+    l_rows = torch.stack([l[b, h, i] for (b, h, i) in rows])
+    check_o(o_rows, o_ref, kind, what)
+    check_lse(l_rows, l_ref, what)
+    return o_ref, l_ref
+
+
+def test_workload2_image_dit():
+    w = W.WORKLOADS[2]
+    x = W.make_inputs(w)
+    q, k, v = (x[n].to(DEV) for n in ("q", "k", "v"))
+    o32, l32 = cp.fwd(q, k, v, scale=w.softmax_scale, out_dtype=torch.float32)
+    o16, l16 = cp.fwd(q, k, v, scale=w.softmax_scale)
+    torch.cuda.synchronize()
+    rows = W.sample_rows(w.B, w.H, w.Sq, 2048, seed=2)
+    _sampled(x["q"], x["k"], x["v"], w.softmax_scale, o32.cpu(), l32.cpu(), rows, "bf16_in", "w2 fp32-O")
+    _sampled(x["q"], x["k"], x["v"], w.softmax_scale, o16.cpu(), l16.cpu(), rows, "bf16_out", "w2 bf16-O")
+
+
+def test_workload3_ring_step():
+    w = W.WORKLOADS[3]
+    x = W.make_inputs(w)
+    q, k, v = (x[n].to(DEV) for n in ("q", "k", "v"))
+    bounds = np.cumsum([0] + x["chunks"])
+    kc = [k[:, a:b].contiguous() for a, b in zip(bounds, bounds[1:])]
+    vc = [v[:, a:b].contiguous() for a, b in zip(bounds, bounds[1:])]
+    o_ring, l_ring = cp.ring_attention(q, kc, vc, scale=w.softmax_scale)
+    o_ring32, l_ring32 = cp.ring_attention(q, kc, vc, scale=w.softmax_scale, acc_dtype=torch.float32)
+    o_one, l_one = cp.fwd(q, k, v, scale=w.softmax_scale, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    rows = W.sample_rows(w.B, w.H, w.Sq, 2048, seed=3)
+    _sampled(x["q"], x["k"], x["v"], w.softmax_scale, o_ring.cpu(), l_ring.cpu(), rows, "bf16_out", "ring bf16")
+    _sampled(x["q"], x["k"], x["v"], w.softmax_scale, o_ring32.cpu(), l_ring32.cpu(), rows, "bf16_in", "ring fp32")
+    _sampled(x["q"], x["k"], x["v"], w.softmax_scale, o_one.cpu(), l_one.cpu(), rows, "bf16_in", "single pass")
+    # whole-tensor property: ring result == single-pass result
+    assert (o_ring32 - o_one).abs().max().item() < 1e-3
+    assert (l_ring32 - l_one).abs().max().item() < 1e-4
+
+
+def test_workload4_ulysses():
+    w = W.WORKLOADS[4]
+    x = W.make_inputs(w)  # per-rank shards [P][S_l][H][D]
+    P = w.P
+    q, k, v = (x[n].to(DEV) for n in ("q", "k", "v"))
+    plan = UlyssesPlan(P, w.Sq // P, w.H * P, w.D)
+    out, lse = plan.run(q, k, v, scale=w.softmax_scale)
+    torch.cuda.synchronize()
+    # the permutes are bit-exact against the oracle's re-partition
+    for name, dev_buf in (("q", plan.qh), ("k", plan.kh), ("v", plan.vh)):
+        np.testing.assert_array_equal(bits(dev_buf).cpu().numpy(),
+                                      ref.seq2head(bits(x[name]).numpy(), P))
+    np.testing.assert_array_equal(bits(out).cpu().numpy(),
+                                  ref.head2seq(bits(plan.oh).cpu().numpy(), P))
+    # attention: single-device semantics -- full sequence = shards in rank order
+    S_l, H = w.Sq // P, w.H * P
+    full = lambda t: t.reshape(1, P * S_l, H, w.D)
+    rows = W.sample_rows(1, H, P * S_l, 4096, seed=4)
+    o_ref, l_ref = ref.attention_rows(full(x["q"]), full(x["k"]), full(x["v"]), w.softmax_scale, rows)
+    out_c, lse_c = out.cpu(), lse.cpu()
+    o_rows = torch.stack([out_c[t // S_l, t % S_l, h] for (_, h, t) in rows])
+    l_rows = torch.stack([lse_c[h // w.H, h % w.H, t] for (_, h, t) in rows])
+    check_o(o_rows, o_ref, "bf16_out", "ulysses O")
+    check_lse(l_rows, l_ref, "ulysses LSE")
+
+
+def test_workload5_long_joint_sigma3():
+    w = W.WORKLOADS[5]
+    x = W.make_inputs(w)
+    q, k, v = (x[n].to(DEV) for n in ("q", "k", "v"))
+    o32, l32 = cp.fwd(q, k, v, scale=w.softmax_scale, out_dtype=torch.float32)
+    o16, _ = cp.fwd(q, k, v, scale=w.softmax_scale)
+    torch.cuda.synchronize()
+    rows = W.sample_rows(w.B, w.H, w.Sq, 4096, seed=5)
+    o_ref, _ = _sampled(x["q"], x["k"], x["v"], w.softmax_scale, o32.cpu(), l32.cpu(), rows,
+                        "bf16_in", "w5 fp32-O")
+    o16c = o16.cpu()
+    check_o(torch.stack([o16c[b, i, h] for (b, h, i) in rows]), o_ref, "bf16_out", "w5 bf16-O")
+
+
+# ----------------------------------------------------------------------------- bounded waits
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    assert cp.device_error() == 0
+    cp.selftest_wait_timeout(1_000_000)  # ~0.5 ms of SM cycles, nothing ever arrives
+    assert cp.device_error() == cp._binding.ERR_DEVICE_TIMEOUT
+    assert cp.device_error() == 0  # the word was cleared
+    q, k, v = (t.to(DEV) for t in W.random_case(1, 1, 1, 64, 64, 128))
+    o, l = cp.fwd(q, k, v)
+    torch.cuda.synchronize()
+    check_o(o, ref.attention(q.cpu(), k.cpu(), v.cpu(), 1 / math.sqrt(128))[0], "bf16_out", "after")
