@@ -1,0 +1,444 @@
+#!/usr/bin/env python
+"""Benchmark of the per-rank context-parallel attention hot path on B200.
+
+One step = one pass of the Ulysses path over the S=44160 video-latent workload:
+P=8 virtual ranks x [5520 tokens][16 heads][128] bf16 Q/K/V -> 3 seq2head permutes ->
+non-causal attention over B=8 head groups x 2 heads x S=44160 x D=128 (tcgen05 kernel)
+-> head2seq permute.  The metric is attention TFLOPS (4*B*H*S^2*D per step) over the
+whole step; the attention kernel's own roofline, the permutes' and the (O, LSE) merge's
+HBM rooflines and an end-to-end number through host buffers are reported beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs its own replica (weak scaling, no data-path
+collective); the timed region is bracketed by barriers and the max over ranks is used.
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from context_long_sequence_non_b200 import workloads as W  # noqa: E402
+
+METRIC = "non-causal bf16 attention TFLOPS at S=44160 on 1 B200; % of dense BF16 peak"
+UNIT = "TFLOP/s"
+WORKLOAD = W.WORKLOADS[4]
+L2_NOTE = ("inputs larger than L2: each step streams 543 MB of Q/K/V shards plus 724 MB of "
+           "permute traffic through the 126 MB L2")
+
+
+def workload_config():
+    w = WORKLOAD
+    return {
+        "workload": (f"ulysses-cp8-s44160: P=8 virtual ranks x [5520 tokens][16 heads][128] bf16 "
+                     f"Q/K/V, 3x seq2head + non-causal attention (8 head groups x 2 heads, "
+                     f"S=44160, D=128, fp32 accumulate, bf16 O + fp32 LSE) + head2seq"),
+        "B": w.B, "H": w.H, "S": w.Sq, "D": w.D, "P": w.P,
+        "inputs": "iid N(0,1), torch.Generator seed 4000, rounded to bf16",
+        "l2": L2_NOTE,
+    }
+
+
+# --------------------------------------------------------------------------- distributed
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_group(world, backend):
+    if world <= 1:
+        return None
+    import datetime
+
+    import torch.distributed as dist
+
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def aggregate(dist, elapsed_ms: float, units: float, device=None):
+    """Max of the timed region over ranks and the sum of the work units of all ranks."""
+    if dist is None:
+        return elapsed_ms, units
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
+    u = torch.tensor([units], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+# --------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, path: str | None = None):
+        self.gpu_index, self.proc, self.path = gpu_index, None, path
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        if self.path:
+            with open(self.path, "w") as f:
+                f.write(out)
+        sm, mx, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+                power.append(float(r[3]))
+            except ValueError:
+                continue
+            for n, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# --------------------------------------------------------------------------- peaks
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# --------------------------------------------------------------------------- our arm
+
+
+def run_ours(args, world, rank, local):
+    import context_long_sequence_non_b200 as cp
+    from context_long_sequence_non_b200 import _binding as Bd
+    from context_long_sequence_non_b200.paths import UlyssesPlan
+
+    torch.cuda.set_device(local)
+    dist = init_group(world, "nccl")
+    dev = torch.device("cuda", local)
+    w = WORKLOAD
+    P, S_l, H = w.P, w.Sq // w.P, w.H * w.P
+    x = W.make_inputs(w)
+    global _INPUTS
+    _INPUTS = x
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    plan = UlyssesPlan(P, S_l, H, w.D, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flops = w.attn_flops
+    launches_per_step = 5
+
+    def step(ev_attn=None):
+        cp.seq2head(q, P, out=plan.qh)
+        cp.seq2head(k, P, out=plan.kh)
+        cp.seq2head(v, P, out=plan.vh)
+        if ev_attn is not None:
+            ev_attn[0].record(stream)
+        cp.fwd(plan.qh, plan.kh, plan.vh, out=plan.oh, lse=plan.lse, scale=w.softmax_scale)
+        if ev_attn is not None:
+            ev_attn[1].record(stream)
+        cp.head2seq(plan.oh, P, out=plan.out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if Bd.device_error() != 0:
+        raise RuntimeError("bounded wait ran out during warm-up")
+
+    clocks = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
+                          if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else None)
+    attn_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)  # let the sampler take its first reading
+    t0.record(stream)
+    for i in range(args.steps):
+        step(attn_events[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if dist is not None:
+        dist.barrier()
+    elapsed_ms = t0.elapsed_time(t1)
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in attn_events)
+    if Bd.device_error() != 0:
+        raise RuntimeError("bounded wait ran out during the timed region")
+    max_ms, total_flops = aggregate(dist, elapsed_ms, flops * args.steps,
+                                    device=dev if dist is not None else None)
+
+    # ---- auxiliary HBM-bound kernels, timed alone (L2 flushed before each launch)
+    aux = aux_kernels(cp, w, q, plan, dev, stream)
+
+    # ---- end to end through the public API with host buffers
+    e2e = e2e_run(cp, UlyssesPlan, w, x, dev, stream, args)
+
+    peaks = measured_peaks()
+    value = total_flops / (max_ms * 1e-3) / 1e12
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    long_run = max_ms > 1000.0
+    peak = peaks["bf16_tflops_sustained"] if long_run else peaks["bf16_tflops"]
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(max_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(),
+        "frac_of_dense_bf16_peak": round(value / peak, 4),
+        "roofline": {
+            "bound": "tensor", "kernel": "attn_fwd_sm100_kernel<128,false>",
+            "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4),
+            "peak_kind": (f"{peaks['source']} cuBLAS bf16 "
+                          f"{'sustained' if long_run else 'burst'}"),
+            "algorithmic_flops_per_launch": flops,
+            "avg_launch_ms": round(attn_ms, 4), "traffic": None,
+        },
+        "aux": aux,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def flush_l2(buf):
+    buf.zero_()
+
+
+def aux_kernels(cp, w, q, plan, dev, stream):
+    """seq2head / head2seq / merge alone: achieved HBM GB/s (bytes read + written once)."""
+    peaks = measured_peaks()
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)  # 4x the 126 MB L2
+    out = {}
+
+    def timed(fn, reps=10):
+        ts = []
+        for _ in range(reps):
+            flush_l2(flush)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    P = w.P
+    tensor_bytes = q.numel() * q.element_size()
+    ms = timed(lambda: cp.seq2head(q, P, out=plan.qh))
+    out["seq2head"] = {"ms": round(ms, 4), "bytes": 2 * tensor_bytes,
+                       "GB/s": round(2 * tensor_bytes / ms / 1e6, 1),
+                       "frac_of_hbm": round(2 * tensor_bytes / ms / 1e6 / peaks["hbm_gbs"], 4)}
+    ms = timed(lambda: cp.head2seq(plan.oh, P, out=plan.out))
+    out["head2seq"] = {"ms": round(ms, 4), "bytes": 2 * tensor_bytes,
+                       "GB/s": round(2 * tensor_bytes / ms / 1e6, 1),
+                       "frac_of_hbm": round(2 * tensor_bytes / ms / 1e6 / peaks["hbm_gbs"], 4)}
+    # ring-step merge on one rank's partial: [5520][16][128] bf16 + LSE [16][5520]
+    S, Hm, D = 5520, 16, 128
+    g = torch.Generator(device="cpu").manual_seed(31)
+    oa = torch.randn(1, S, Hm, D, generator=g).to(torch.bfloat16).to(dev)
+    ob = torch.randn(1, S, Hm, D, generator=g).to(torch.bfloat16).to(dev)
+    la = torch.randn(1, Hm, S, generator=g).to(dev)
+    lb = torch.randn(1, Hm, S, generator=g).to(dev)
+    om, lm = torch.empty_like(oa), torch.empty_like(la)
+    ms = timed(lambda: cp.merge(oa, la, ob, lb, out=om, lse=lm))
+    mbytes = 3 * oa.numel() * 2 + 3 * la.numel() * 4
+    out["merge"] = {"ms": round(ms, 4), "bytes": mbytes, "GB/s": round(mbytes / ms / 1e6, 1),
+                    "frac_of_hbm": round(mbytes / ms / 1e6 / peaks["hbm_gbs"], 4),
+                    "shape": "[1][5520][16][128] bf16 x3 + LSE [1][16][5520] f32 x3"}
+    out["hbm_peak_gbs"] = peaks["hbm_gbs"]
+    out["l2"] = "512 MB buffer written before each launch (L2 flushed)"
+    return out
+
+
+def e2e_run(cp, UlyssesPlan, w, x, dev, stream, args):
+    """Same metric through the public API with pinned host buffers: H2D of the step's
+    Q/K/V shards and D2H of O and LSE inside the timed region."""
+    P, S_l, H = w.P, w.Sq // w.P, w.H * w.P
+    hq, hk, hv = (x[n].pin_memory() for n in ("q", "k", "v"))
+    plan = UlyssesPlan(P, S_l, H, w.D, device=dev)
+    dq, dk, dv = (torch.empty_like(hq, device=dev) for _ in range(3))
+    ho = torch.empty(plan.out.shape, dtype=plan.out.dtype).pin_memory()
+    hl = torch.empty(plan.lse.shape, dtype=plan.lse.dtype).pin_memory()
+
+    def step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        plan.run(dq, dk, dv, scale=w.softmax_scale)
+        ho.copy_(plan.out, non_blocking=True)
+        hl.copy_(plan.lse, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(dev)
+    n = max(3, min(args.steps, 10))
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b) / n
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+    return {"value": round(w.attn_flops / (ms * 1e-3) / 1e12, 2), "unit": UNIT,
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": n}
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+
+def oracle_sample(n_rows, seed):
+    """The fp64 oracle on ``n_rows`` sampled query rows of the Ulysses workload (each row
+    attends over all 44160 keys of its head).  Returns (seconds, flops, cores)."""
+    import oracle
+
+    cores = oracle.set_threads()
+    w = WORKLOAD
+    x = _oracle_inputs()
+    S_l, H = w.Sq // w.P, w.H * w.P
+    full = lambda t: t.reshape(1, w.P * S_l, H, w.D)
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    hs = torch.randint(0, H, (n_rows,), generator=g).tolist()
+    ts = torch.randint(0, w.Sq, (n_rows,), generator=g).tolist()
+    rows = [(0, h, t) for h, t in zip(hs, ts)]
+    t = time.perf_counter()
+    oracle.attention_rows(full(x["q"]), full(x["k"]), full(x["v"]), w.softmax_scale, rows)
+    dt = time.perf_counter() - t
+    return dt, 4.0 * len(rows) * w.Skv * w.D, cores
+
+
+_INPUTS = None
+
+
+def _oracle_inputs():
+    global _INPUTS
+    if _INPUTS is None:
+        _INPUTS = W.make_inputs(WORKLOAD)
+    return _INPUTS
+
+
+def cpu_baseline(budget_s=15.0):
+    n, spent, flops, cores = 64, 0.0, 0.0, 1
+    rounds = 0
+    while spent < budget_s and rounds < 12:
+        dt, f, cores = oracle_sample(n, seed=100 + rounds)
+        spent += dt
+        flops += f
+        rounds += 1
+        if dt < budget_s / 4:
+            n *= 2
+    return {"value": round(flops / spent / 1e12, 6), "unit": UNIT, "cores": cores,
+            "kind": "oracle",
+            "sample": (f"{int(flops / (4 * WORKLOAD.Skv * WORKLOAD.D))} query rows of the "
+                       f"S=44160 Ulysses workload (each over all 44160 keys), fp64 NumPy/BLAS, "
+                       f"{spent:.1f} s")}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return  # the CPU oracle arm runs on rank 0 only
+    rows_per_step = 128
+    for i in range(args.warmup):
+        oracle_sample(rows_per_step, seed=1 + i)
+    tot_t, tot_f, cores = 0.0, 0.0, 1
+    for i in range(args.steps):
+        dt, f, cores = oracle_sample(rows_per_step, seed=1000 + i)
+        tot_t += dt
+        tot_f += f
+    value = tot_f / tot_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(tot_t / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(),
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"{rows_per_step} query rows per step of the S=44160 Ulysses "
+                                   f"workload, each over all 44160 keys, fp64 NumPy/BLAS"},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps")
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+    else:
+        run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -123,9 +123,9 @@ int cpattn_fwd(const void* q, const void* k, const void* v, void* out, float* ls
         !encode_bshd_bf16(&tv, v, B, Skv, H, D))
       return CPATTN_ERR_CUDA;
     const float scale_log2 = float(double(scale) * 1.4426950408889634074);
-    return cuda_status(cpattn::launch_attn_fwd_sm100(tq, tk, tv, out, lse, B, H, Sq, Skv, D,
-                                                     scale_log2, out_dtype == CPATTN_F32, err,
-                                                     cpattn::kDefaultWaitLimit, st));
+    return cuda_status(cpattn::launch_attn_fwd_sm100(
+        tq, tk, tv, out, lse, B, H, Sq, Skv, D, scale_log2, cpattn::kRescaleLog2,
+        out_dtype == CPATTN_F32, err, cpattn::kDefaultWaitLimit, st));
   }
   // fp32 inputs: CUDA-core kernel
   return cuda_status(cpattn::launch_attn_fwd_f32(

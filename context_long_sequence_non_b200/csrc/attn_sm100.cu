@@ -16,9 +16,11 @@
 // bf16 pairs) | O0 | O1 (D fp32 columns each).  S = Q K^T runs smem x smem; O += P V
 // takes P from TMEM and V from smem (MN-major).  While softmax works on one Q tile the
 // tensor core runs the other tile's MMAs (ping-pong), and TMA prefetches ahead.
-// Softmax works in base 2: x = s * scale * log2(e); the running max is only raised when
-// it grows by more than kRescaleLog2 (a stale max is exact because the final
-// normalisation uses the same max); O is rescaled in TMEM by the softmax warps then.
+// Softmax works in base 2: x = s * scale * log2(e).  The running max is raised when a
+// block's row max exceeds it by more than `rescale_log2` (0 = an exact running max; a
+// stale max is still exact in real arithmetic because the final normalisation uses the
+// same max, but with an exact max the dominant key's P is exactly 1 in bf16).  O is
+// rescaled in TMEM by the softmax warps when the max moves.
 // Every wait is bounded (mbar_wait): a stalled pipeline sets the device error word and
 // the CTA drains and exits instead of hanging.
 #include <cuda_runtime.h>
@@ -35,7 +37,6 @@ constexpr int kSlots = 4;        // K/V ring slots (K_j and V_j alternate)
 constexpr int kThreads = 384;
 constexpr int kWarpProducer = 8;
 constexpr int kWarpMma = 9;
-constexpr float kRescaleLog2 = 8.0f;  // raise the running max only past a 2^8 growth
 constexpr uint32_t kTmemCols = 512;
 
 template <int D>
@@ -68,7 +69,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, void* __restrict__ out,
                           float* __restrict__ lse, int H, int Sq, int Skv, float scale_log2,
-                          int* err, long long wait_limit) {
+                          float rescale_log2, int* err, long long wait_limit) {
   using G = Geometry<D>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ Barriers bars;
@@ -161,7 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (j == 0) {
         m = m_tile;
       } else {
-        const bool grow = m_tile > m + kRescaleLog2;
+        const bool grow = m_tile > m + rescale_log2;
         rescale = __any_sync(0xffffffffu, grow);
         if (rescale) {
           const float m_new = grow ? m_tile : m;
@@ -365,8 +366,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, bool kOutF32>
 cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* out,
-                   float* lse, int B, int H, int Sq, int Skv, float scale_log2, int* err,
-                   long long wait_limit, cudaStream_t stream) {
+                   float* lse, int B, int H, int Sq, int Skv, float scale_log2,
+                   float rescale_log2, int* err, long long wait_limit, cudaStream_t stream) {
   using G = Geometry<D>;
   auto kernel = attn_fwd_sm100_kernel<D, kOutF32>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -374,7 +375,7 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   if (e != cudaSuccess) return e;
   dim3 grid((Sq + 2 * kBlockM - 1) / (2 * kBlockM), H, B);
   kernel<<<grid, kThreads, G::kDynSmem, stream>>>(tq, tk, tv, out, lse, H, Sq, Skv, scale_log2,
-                                                   err, wait_limit);
+                                                   rescale_log2, err, wait_limit);
   return cudaGetLastError();
 }
 
@@ -382,18 +383,19 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
 
 cudaError_t launch_attn_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
                                   const CUtensorMap& tv, void* out, float* lse, int B, int H,
-                                  int Sq, int Skv, int D, float scale_log2, bool out_f32, int* err,
-                                  long long wait_limit, cudaStream_t stream) {
+                                  int Sq, int Skv, int D, float scale_log2, float rescale_log2,
+                                  bool out_f32, int* err, long long wait_limit,
+                                  cudaStream_t stream) {
   if (D == 128) {
-    return out_f32 ? launch<128, true>(tq, tk, tv, out, lse, B, H, Sq, Skv, scale_log2, err,
-                                       wait_limit, stream)
-                   : launch<128, false>(tq, tk, tv, out, lse, B, H, Sq, Skv, scale_log2, err,
-                                        wait_limit, stream);
+    return out_f32 ? launch<128, true>(tq, tk, tv, out, lse, B, H, Sq, Skv, scale_log2,
+                                       rescale_log2, err, wait_limit, stream)
+                   : launch<128, false>(tq, tk, tv, out, lse, B, H, Sq, Skv, scale_log2,
+                                        rescale_log2, err, wait_limit, stream);
   }
-  return out_f32 ? launch<64, true>(tq, tk, tv, out, lse, B, H, Sq, Skv, scale_log2, err,
-                                    wait_limit, stream)
-                 : launch<64, false>(tq, tk, tv, out, lse, B, H, Sq, Skv, scale_log2, err,
-                                     wait_limit, stream);
+  return out_f32 ? launch<64, true>(tq, tk, tv, out, lse, B, H, Sq, Skv, scale_log2,
+                                    rescale_log2, err, wait_limit, stream)
+                 : launch<64, false>(tq, tk, tv, out, lse, B, H, Sq, Skv, scale_log2,
+                                     rescale_log2, err, wait_limit, stream);
 }
 
 }  // namespace cpattn

@@ -14,8 +14,13 @@ constexpr long long kDefaultWaitLimit = 2000000000LL;
 // tensors with a 64 x 1 x 128 x 1 box and 128-byte swizzle.
 cudaError_t launch_attn_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
                                   const CUtensorMap& tv, void* out, float* lse, int B, int H,
-                                  int Sq, int Skv, int D, float scale_log2, bool out_f32, int* err,
-                                  long long wait_limit, cudaStream_t stream);
+                                  int Sq, int Skv, int D, float scale_log2, float rescale_log2,
+                                  bool out_f32, int* err, long long wait_limit,
+                                  cudaStream_t stream);
+
+// Running-max policy of the tensor-core kernel: 0 = exact running max (the dominant key's
+// P is exactly 1, so its bf16 rounding costs nothing).
+constexpr float kRescaleLog2 = 0.0f;
 
 // fp32 CUDA-core attention, D <= 256.
 cudaError_t launch_attn_fwd_f32(const float* q, const float* k, const float* v, void* out,
