@@ -217,11 +217,13 @@ def run_ours(args, world, rank, local):
     max_ms, total_flops = aggregate(dist, elapsed_ms, flops * args.steps,
                                     device=dev if dist is not None else None)
 
-    # ---- auxiliary HBM-bound kernels, timed alone (L2 flushed before each launch)
-    aux = aux_kernels(cp, w, q, plan, dev, stream)
-
-    # ---- end to end through the public API with host buffers
-    e2e = e2e_run(cp, UlyssesPlan, w, x, dev, stream, args)
+    if args.profile:  # profiler runs: the timed steps only, nothing else launched
+        aux, e2e = None, None
+    else:
+        # ---- auxiliary HBM-bound kernels, timed alone (L2 flushed before each launch)
+        aux = aux_kernels(cp, w, q, plan, dev, stream)
+        # ---- end to end through the public API with host buffers
+        e2e = e2e_run(cp, UlyssesPlan, w, x, dev, stream, args)
 
     peaks = measured_peaks()
     value = total_flops / (max_ms * 1e-3) / 1e12
@@ -249,7 +251,7 @@ def run_ours(args, world, rank, local):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not (args.no_cpu_baseline or args.profile):
         line["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -430,6 +432,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="for profiler captures: run only warm-up + timed steps (no aux "
+                         "kernels, no end-to-end pass, no CPU baseline)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
