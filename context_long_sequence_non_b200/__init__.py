@@ -20,6 +20,7 @@ from ._binding import (  # noqa: F401
     lib,
     library_path,
     merge,
+    selftest_exp2,
     selftest_wait_timeout,
     seq2head,
     status_str,

@@ -55,8 +55,10 @@ def lib() -> ctypes.CDLL:
             L.cpattn_device_error.argtypes = []
             L.cpattn_selftest_wait_timeout.argtypes = [ll, vp]
             L.cpattn_version.argtypes = []
+            L.cpattn_selftest_exp2.argtypes = [vp, vp, i, vp]
             for name in ("cpattn_fwd", "cpattn_merge", "cpattn_seq2head", "cpattn_head2seq",
-                         "cpattn_device_error", "cpattn_selftest_wait_timeout", "cpattn_version"):
+                         "cpattn_device_error", "cpattn_selftest_wait_timeout", "cpattn_version",
+                         "cpattn_selftest_exp2"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -175,6 +177,16 @@ def device_error() -> int:
 def selftest_wait_timeout(limit_cycles: int, stream=None):
     _check(lib().cpattn_selftest_wait_timeout(int(limit_cycles), _stream(stream)),
            "cpattn_selftest_wait_timeout")
+
+
+def selftest_exp2(t, out=None, stream=None):
+    """The attention kernel's FMA-pipe 2^t on a float32 CUDA tensor (test hook)."""
+    if out is None:
+        out = torch.empty_like(t)
+    _need_cuda(t, out)
+    _check(lib().cpattn_selftest_exp2(_ptr(t), _ptr(out), t.numel(), _stream(stream)),
+           "cpattn_selftest_exp2")
+    return out
 
 
 def version() -> int:

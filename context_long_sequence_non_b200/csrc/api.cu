@@ -138,7 +138,7 @@ int cpattn_merge(const void* o_a, const float* lse_a, const void* o_b, const flo
   if (B < 1 || H < 1 || S < 1 || D < 1) return CPATTN_ERR_SHAPE;
   const int es = elem_size(dtype);
   if (es == 0) return CPATTN_ERR_UNSUPPORTED;
-  if ((D * es) % 16 != 0) return CPATTN_ERR_SHAPE;
+  if ((D * es) % 16 != 0 || D * es > 4096) return CPATTN_ERR_SHAPE;
   if (!o_a || !lse_a || !o_b || !lse_b || !o || !lse) return CPATTN_ERR_NULL;
   if (!aligned(o_a, 16) || !aligned(o_b, 16) || !aligned(o, 16) || !aligned(lse_a, 4) ||
       !aligned(lse_b, 4) || !aligned(lse, 4))
@@ -204,6 +204,14 @@ int cpattn_selftest_wait_timeout(long long limit_cycles, cpattn_stream_t stream)
   if (err == nullptr) return CPATTN_ERR_CUDA;
   return cuda_status(cpattn::launch_wait_timeout_selftest(err, limit_cycles,
                                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int cpattn_selftest_exp2(const float* t, float* out, int n, cpattn_stream_t stream) {
+  if (n < 1) return CPATTN_ERR_SHAPE;
+  if (t == nullptr || out == nullptr) return CPATTN_ERR_NULL;
+  if (!aligned(t, 4) || !aligned(out, 4)) return CPATTN_ERR_ALIGN;
+  return cuda_status(
+      cpattn::launch_exp2_poly_selftest(t, out, n, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -37,7 +37,17 @@ constexpr int kSlots = 4;        // K/V ring slots (K_j and V_j alternate)
 constexpr int kThreads = 384;
 constexpr int kWarpProducer = 8;
 constexpr int kWarpMma = 9;
+// Register split (setmaxnreg): the CTA launches with 168 x 384 = 64512 registers; the two
+// softmax warpgroups take 216 each per thread and the producer/MMA warpgroup 72:
+// 2 x 128 x 216 + 128 x 72 = 64512 (no spills at this split; 56 spills in the issuer).
+constexpr uint32_t kRegsLaunch = 168, kRegsSoftmax = 216, kRegsOther = 72;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kRegsLaunch * kThreads,
+              "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
+// exp2 work split: of every 8 column pairs, this many go through the FMA-pipe polynomial
+// and the rest through the special-function unit (ex2), which would otherwise be
+// co-critical with the tensor core (one ex2 per score, 16 per clock per SM).
+constexpr int kPolyPairs = 2;
 
 template <int D>
 struct Geometry {
@@ -118,6 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 8) {
     // ------------------------------------------------------------------ softmax warps
+    regs_inc<kRegsSoftmax>();
     const int tile = warp >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // row within the Q tile == TMEM lane
@@ -136,12 +147,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
 
       float x[kBlockN];
+      {
+        uint32_t r[kBlockN];
+        tmem_ld128(t_s, r);  // the whole S row, one wait
 #pragma unroll
-      for (int c = 0; c < kBlockN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(t_s + c * 32, r);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(r[e]);
+        for (int c = 0; c < kBlockN; ++c) x[c] = __uint_as_float(r[c]);
       }
       const int valid = Skv - j * kBlockN;  // keys of this tile inside the sequence
       if (valid < kBlockN) {
@@ -149,14 +159,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < kBlockN; ++c)
           if (c >= valid) x[c] = -INFINITY;
       }
-      // row maximum of the scaled logits (scale > 0 is a precondition of the call)
-      float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
+      // row maximum of the raw logits (scale > 0 is a precondition of the call): a tree of
+      // three-input max, 64 instructions and 5 levels deep (a chain would be latency-bound)
+      float mx;
+      {
+        float l1[44];
 #pragma unroll
-      for (int c = 4; c < kBlockN; c += 4) {
-        mx0 = fmaxf(mx0, x[c]); mx1 = fmaxf(mx1, x[c + 1]);
-        mx2 = fmaxf(mx2, x[c + 2]); mx3 = fmaxf(mx3, x[c + 3]);
+        for (int i = 0; i < 42; ++i) l1[i] = max3(x[3 * i], x[3 * i + 1], x[3 * i + 2]);
+        l1[42] = x[126];
+        l1[43] = x[127];
+        float l2[16];
+#pragma unroll
+        for (int i = 0; i < 14; ++i) l2[i] = max3(l1[3 * i], l1[3 * i + 1], l1[3 * i + 2]);
+        l2[14] = l1[42];
+        l2[15] = l1[43];
+        float l3[6];
+#pragma unroll
+        for (int i = 0; i < 5; ++i) l3[i] = max3(l2[3 * i], l2[3 * i + 1], l2[3 * i + 2]);
+        l3[5] = l2[15];
+        mx = fmaxf(max3(l3[0], l3[1], l3[2]), max3(l3[3], l3[4], l3[5]));
       }
-      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * scale_log2;
+      const float m_tile = mx * scale_log2;
       float alpha = 1.0f;
       bool rescale = false;
       if (j == 0) {
@@ -171,35 +194,50 @@ __global__ void __launch_bounds__(kThreads, 1)
           l *= alpha;
         }
       }
-      // p = 2^(x - m), rounded to bf16 for the PV product, written over S as bf16 pairs
-      const float neg_m = -m;
-      float sum0 = 0.f, sum1 = 0.f;
+      // p = 2^(x * scale_log2 - m): most pairs on the special-function unit, kPolyPairs of
+      // every 8 pairs on the FMA pipe (exp2_poly2); p rounded to bf16 for the PV product and
+      // written over S as bf16 pairs; the row sum keeps the unrounded fp32 p
+      const float2 sl2 = make_float2(scale_log2, scale_log2);
+      const float2 nm2 = make_float2(-m, -m);
+      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const float p0 = ex2(fmaf(x[half * 64 + 2 * e], scale_log2, neg_m));
-          const float p1 = ex2(fmaf(x[half * 64 + 2 * e + 1], scale_log2, neg_m));
-          sum0 += p0;
-          sum1 += p1;
-          pk[e] = pack_bf16x2(p0, p1);
+          const int c = half * 64 + 2 * e;
+          const float2 t = ffma2(make_float2(x[c], x[c + 1]), sl2, nm2);
+          float2 pv;
+          if ((e & 7) >= 8 - kPolyPairs) {
+            pv = exp2_poly2(t);
+          } else {
+            pv.x = ex2(t.x);
+            pv.y = ex2(t.y);
+          }
+          if (e & 1) acc1 = fadd2(acc1, pv);
+          else acc0 = fadd2(acc0, pv);
+          pk[e] = pack_bf16x2(pv.x, pv.y);
         }
         tmem_st32(t_s + half * 32, pk);
       }
-      l += sum0 + sum1;
+      const float2 acc = fadd2(acc0, acc1);
+      l += acc.x + acc.y;
       if (rescale) {
         // rescale this warp's O rows by alpha: PV of the previous block has completed
         // (the issuer committed this block's S after it) and the next PV waits for
         // p_full, so nothing else touches O now
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(t_o + c * 32, r);
+        uint32_t r[D];
+        if constexpr (D == 128) tmem_ld128(t_o, r);
+        else tmem_ld64(t_o, r);
+        const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tmem_st32(t_o + c * 32, r);
+        for (int c = 0; c < D; c += 2) {
+          const float2 o = fmul2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), a2);
+          r[c] = __float_as_uint(o.x);
+          r[c + 1] = __float_as_uint(o.y);
         }
+        if constexpr (D == 128) tmem_st128(t_o, r);
+        else tmem_st64(t_o, r);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -249,7 +287,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         lse[(size_t(b) * H + h) * Sq + q] = (m + log2f(l)) * 0.69314718055994530942f;
       }
     }
-  } else if (warp == kWarpProducer) {
+  } else {
+    regs_dec<kRegsOther>();
+  }
+  if (warp == kWarpProducer) {
     // ------------------------------------------------------------------ TMA producer
     if (elect_one()) {
       const uint32_t bar_q = smem_u32(&bars.q_full);

@@ -45,6 +45,9 @@ cudaError_t launch_head2seq(const void* src, void* dst, int P, int S_local, long
 // One CTA waiting on an mbarrier nothing completes, with the attention kernel's bounded wait.
 cudaError_t launch_wait_timeout_selftest(int* err, long long limit, cudaStream_t stream);
 
+// The attention kernel's FMA-pipe 2^t (exp2_poly2) applied to n floats.
+cudaError_t launch_exp2_poly_selftest(const float* t, float* out, int n, cudaStream_t stream);
+
 int sm_count();
 
 }  // namespace cpattn

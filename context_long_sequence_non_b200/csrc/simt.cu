@@ -92,13 +92,13 @@ __global__ void fill_empty_kernel(uint4* out, size_t n_vec, float* lse, size_t n
 }
 
 // ------------------------------------------------------------------ (O, LSE) merge
-// A block takes kRows consecutive (b, s, h) rows: phase 1 turns the two LSEs of each row
-// into weights (and writes the merged LSE), phase 2 streams the O rows as 16-byte vectors.
-// Every O element and every LSE entry is read and written by the same thread, so the
-// merged result may overwrite partial a in place.
-constexpr int kMergeRows = 64;
+// One 16-byte vector of O per thread; a block covers whole (b, s, h) rows (blockDim =
+// rows_per_block x vectors_per_row).  Every thread derives its row's weights from the two
+// LSEs itself (no shared-memory phase), so loads of O and LSE are all in flight at once.
+// The merged LSE is written after a block barrier by the row's first thread: every read of
+// this block's LSE entries precedes every write, and each O vector is read and written by
+// the same thread, so the result may overwrite partial a in place.
 constexpr int kMergeThreads = 256;
-constexpr int kMergeUnroll = 4;
 
 __device__ __forceinline__ void merge_vec_bf16(const uint4& a, const uint4& b, float wa, float wb,
                                                uint4& o) {
@@ -125,58 +125,39 @@ template <bool kBf16>
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
     const uint4* o_a, const float* lse_a, const uint4* o_b, const float* lse_b, uint4* o,
     float* lse, int H, int S, long long n_rows, int vpr) {
-  __shared__ float wa_s[kMergeRows], wb_s[kMergeRows];
-  for (long long r0 = (long long)blockIdx.x * kMergeRows; r0 < n_rows;
-       r0 += (long long)gridDim.x * kMergeRows) {
-    const int rows_here = int(n_rows - r0 < kMergeRows ? n_rows - r0 : kMergeRows);
-    if (threadIdx.x < rows_here) {
-      const long long row = r0 + threadIdx.x;  // (b, s, h), h fastest
-      const int h = int(row % H);
-      const long long bs = row / H;
-      const int s = int(bs % S);
-      const long long b = bs / S;
-      const long long li = (b * H + h) * S + s;
-      const float la = lse_a[li], lb = lse_b[li];
-      const float mx = fmaxf(la, lb);
-      float wa = 0.f, wb = 0.f, L = -INFINITY;
-      if (mx != -INFINITY) {
-        const float ea = expf(la - mx), eb = expf(lb - mx);
-        const float tot = ea + eb;
-        L = mx + logf(tot);
-        wa = ea / tot;
-        wb = eb / tot;
-      }
-      wa_s[threadIdx.x] = wa;
-      wb_s[threadIdx.x] = wb;
-      lse[li] = L;
+  const int rows_per_block = blockDim.x / vpr;
+  const int rl = threadIdx.x / vpr;
+  const int v = threadIdx.x - rl * vpr;
+  const long long row = (long long)blockIdx.x * rows_per_block + rl;  // (b, s, h), h fastest
+  const bool live = rl < rows_per_block && row < n_rows;
+  long long li = 0;
+  float L = -INFINITY;
+  if (live) {
+    const int h = int(row % H);
+    const long long bs = row / H;
+    const int s = int(bs % S);
+    const long long b = bs / S;
+    li = (b * H + h) * S + s;
+    const long long idx = row * vpr + v;
+    const uint4 a = o_a[idx];
+    const uint4 bv = o_b[idx];
+    const float la = lse_a[li], lb = lse_b[li];
+    const float mx = fmaxf(la, lb);
+    float wa = 0.f, wb = 0.f;
+    if (mx != -INFINITY) {
+      const float ea = expf(la - mx), eb = expf(lb - mx);
+      const float tot = ea + eb;
+      L = mx + logf(tot);
+      wa = ea / tot;
+      wb = eb / tot;
     }
-    __syncthreads();
-    const long long base = r0 * vpr;
-    const int n_vec = rows_here * vpr;
-    for (int v0 = threadIdx.x; v0 < n_vec; v0 += kMergeThreads * kMergeUnroll) {
-      uint4 a[kMergeUnroll], bb[kMergeUnroll];
-#pragma unroll
-      for (int u = 0; u < kMergeUnroll; ++u) {
-        const int v = v0 + u * kMergeThreads;
-        if (v < n_vec) {
-          a[u] = o_a[base + v];
-          bb[u] = o_b[base + v];
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kMergeUnroll; ++u) {
-        const int v = v0 + u * kMergeThreads;
-        if (v < n_vec) {
-          const int rl = v / vpr;
-          uint4 r;
-          if (kBf16) merge_vec_bf16(a[u], bb[u], wa_s[rl], wb_s[rl], r);
-          else merge_vec_f32(a[u], bb[u], wa_s[rl], wb_s[rl], r);
-          o[base + v] = r;
-        }
-      }
-    }
-    __syncthreads();
+    uint4 r;
+    if (kBf16) merge_vec_bf16(a, bv, wa, wb, r);
+    else merge_vec_f32(a, bv, wa, wb, r);
+    o[idx] = r;
   }
+  __syncthreads();
+  if (live && v == 0) lse[li] = L;
 }
 
 // ------------------------------------------------------------------ Ulysses permutes
@@ -226,6 +207,17 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const uint4* __re
     for (int u = 0; u < kPermUnroll; ++u)
       if (live[u]) dst[dst_off[u]] = buf[u];
   }
+}
+
+// ------------------------------------------------------------------ exp2 polynomial self-test
+__global__ void exp2_poly_selftest_kernel(const float* __restrict__ t, float* __restrict__ out,
+                                          int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float2 in = make_float2(t[i], i + 1 < n ? t[i + 1] : 0.f);
+  const float2 r = exp2_poly2(in);
+  out[i] = r.x;
+  if (i + 1 < n) out[i + 1] = r.y;
 }
 
 // ------------------------------------------------------------------ bounded-wait self-test
@@ -309,16 +301,17 @@ cudaError_t launch_merge(const void* o_a, const float* lse_a, const void* o_b, c
                          void* o, float* lse, int B, int H, int S, int D, int elem_bytes,
                          cudaStream_t stream) {
   const long long n_rows = (long long)B * S * H;
-  const int vpr = D * elem_bytes / 16;
-  const long long blocks_needed = (n_rows + kMergeRows - 1) / kMergeRows;
-  long long cap = (long long)sm_count() * 8;  // 8 resident 256-thread blocks per SM
-  const long long blocks = blocks_needed < cap ? blocks_needed : cap;
+  const int vpr = D * elem_bytes / 16;  // 16-byte vectors per row (validated: 1..256)
+  const int rows_per_block = vpr >= kMergeThreads ? 1 : kMergeThreads / vpr;
+  const long long blocks = (n_rows + rows_per_block - 1) / rows_per_block;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  const int threads = rows_per_block * vpr;
   if (elem_bytes == 2)
-    merge_kernel<true><<<unsigned(blocks), kMergeThreads, 0, stream>>>(
+    merge_kernel<true><<<unsigned(blocks), threads, 0, stream>>>(
         static_cast<const uint4*>(o_a), lse_a, static_cast<const uint4*>(o_b), lse_b,
         static_cast<uint4*>(o), lse, H, S, n_rows, vpr);
   else
-    merge_kernel<false><<<unsigned(blocks), kMergeThreads, 0, stream>>>(
+    merge_kernel<false><<<unsigned(blocks), threads, 0, stream>>>(
         static_cast<const uint4*>(o_a), lse_a, static_cast<const uint4*>(o_b), lse_b,
         static_cast<uint4*>(o), lse, H, S, n_rows, vpr);
   return cudaGetLastError();
@@ -352,6 +345,12 @@ cudaError_t launch_seq2head(const void* src, void* dst, int P, int S_local, long
 cudaError_t launch_head2seq(const void* src, void* dst, int P, int S_local, long long run_vec,
                             cudaStream_t stream) {
   return launch_permute(false, src, dst, P, S_local, run_vec, stream);
+}
+
+cudaError_t launch_exp2_poly_selftest(const float* t, float* out, int n, cudaStream_t stream) {
+  const int pairs = (n + 1) / 2;
+  exp2_poly_selftest_kernel<<<(pairs + 255) / 256, 256, 0, stream>>>(t, out, n);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_wait_timeout_selftest(int* err, long long limit, cudaStream_t stream) {

@@ -97,7 +97,8 @@ CPATTN_API int cpattn_fwd(const void* q, const void* k, const void* v, void* out
  * o_a, o_b, o : [B][S][H][D] in `dtype` (BF16 or F32); math in fp32.
  * lse_a, lse_b, lse : [B][H][S] float32.
  * o may alias o_a and lse may alias lse_a (in-place accumulate); no other overlap.
- * D must be a multiple of 8 (BF16) or 4 (F32) so rows move as 16-byte vectors.
+ * D must be a multiple of 8 (BF16) or 4 (F32) so rows move as 16-byte vectors, and a
+ * row must fit in 4096 bytes (D <= 2048 BF16, 1024 F32).
  * Errors: CPATTN_ERR_NULL, _SHAPE, _ALIGN, _UNSUPPORTED (dtype), _CUDA.
  */
 CPATTN_API int cpattn_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
@@ -149,6 +150,16 @@ CPATTN_API int cpattn_device_error(void);
  * Errors: CPATTN_ERR_SHAPE (limit out of range), _CUDA.
  */
 CPATTN_API int cpattn_selftest_wait_timeout(long long limit_cycles, cpattn_stream_t stream);
+
+/*
+ * cpattn_selftest_exp2 -- evaluates, on the device, the polynomial 2^t the attention
+ * kernel uses for a fixed share of its softmax exponentials (Cody-Waite range reduction
+ * t = n + f, |f| <= 1/2, then a degree-3 polynomial with constant term exactly 1, fitted
+ * by csrc/gen_exp2_poly.py; relative error <= 1.02e-4 for -125 <= t <= 0; t below -125
+ * returns 2^-125).  t, out: n device floats.  For tests against the error bound.
+ * Errors: CPATTN_ERR_SHAPE (n < 1), _NULL, _ALIGN, _CUDA.
+ */
+CPATTN_API int cpattn_selftest_exp2(const float* t, float* out, int n, cpattn_stream_t stream);
 
 /* ABI version: (major << 16) | minor. */
 CPATTN_API int cpattn_version(void);

@@ -83,6 +83,7 @@ def test_merge_argument_errors(L):
 
     assert merge(S=0) == B.ERR_SHAPE
     assert merge(D=12) == B.ERR_SHAPE  # 24 bytes: not a whole number of 16-byte vectors
+    assert merge(D=2056) == B.ERR_SHAPE  # a row longer than 4096 bytes
     assert merge(dt=5) == B.ERR_UNSUPPORTED
     assert merge(ptrs=[None] + base[1:]) == B.ERR_NULL
     assert merge(ptrs=base[:4] + [vp(FAKE + 0x400008)] + base[5:]) == B.ERR_ALIGN

@@ -103,7 +103,9 @@ def _check_merge(o, l, oa, la, ob, lb, dt, what):
                                               (1, 5520, 16, 128, torch.bfloat16, 0.0),
                                               (2, 19, 2, 32, torch.float32, 0.0),
                                               (1, 300, 4, 128, torch.bfloat16, 0.3),
-                                              (1, 64, 2, 8, torch.float32, 0.5)])
+                                              (1, 64, 2, 8, torch.float32, 0.5),
+                                              (1, 50, 3, 24, torch.bfloat16, 0.1),
+                                              (1, 9, 2, 1024, torch.float32, 0.0)])
 def test_merge_matches_oracle(Bn, S, H, D, dt, empty):
     oa, la, ob, lb = _rand_partials(S + D, Bn, S, H, D, dt, empty)
     o, l = cp.merge(oa.to(DEV), la.to(DEV), ob.to(DEV), lb.to(DEV))
@@ -314,6 +316,20 @@ def test_workload5_long_joint_sigma3():
                         "bf16_in", "w5 fp32-O")
     o16c = o16.cpu()
     check_o(torch.stack([o16c[b, i, h] for (b, h, i) in rows]), o_ref, "bf16_out", "w5 bf16-O")
+
+
+# ----------------------------------------------------------------------------- exp2 polynomial
+
+
+def test_exp2_polynomial_within_its_bound():
+    t = torch.cat([torch.linspace(-125.0, 0.0, 1_000_001), torch.tensor([0.0, -0.5, -0.25, -1e-7])])
+    out = cp.selftest_exp2(t.to(DEV)).cpu().double().numpy()
+    ref_ = np.exp2(t.double().numpy())
+    rel = np.abs(out / ref_ - 1.0)
+    assert rel.max() <= 1.05e-4, rel.max()
+    assert out[-4] == 1.0  # t = 0 (the row maximum) is exact
+    low = cp.selftest_exp2(torch.tensor([-126.0, -1e4, -math.inf], device=DEV)).cpu()
+    assert torch.all(low == 2.0 ** -125)
 
 
 # ----------------------------------------------------------------------------- bounded waits
