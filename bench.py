@@ -90,9 +90,9 @@ def aggregate(dist, elapsed_ms: float, units: float, device=None):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+    """nvidia-smi clocks and throttle reasons sampled every 50 ms during the timed region."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -103,12 +103,13 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def stop(self, t_begin: float | None = None, t_end: float | None = None):
+        """Stop sampling; summarise the samples taken inside [t_begin, t_end] (epoch s)."""
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -121,10 +122,15 @@ class ClockSampler:
         if self.path:
             with open(self.path, "w") as f:
                 f.write(out)
+        import datetime
+
         sm, mx, reasons, power = [], None, set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
             try:
+                ts = datetime.datetime.strptime(r[0].strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                if t_begin is not None and not (t_begin <= ts <= t_end):
+                    continue
                 sm.append(float(r[1]))
                 mx = float(r[2])
                 power.append(float(r[3]))
@@ -134,8 +140,9 @@ class ClockSampler:
                 if val.strip().lower() == "active":
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm),
-                "power_w_max": max(power) if power else None}
+                "sm_mhz_min": min(sm) if sm else None, "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None,
+                "window": "samples inside the timed region"}
 
 
 # --------------------------------------------------------------------------- peaks
@@ -201,13 +208,15 @@ def run_ours(args, world, rank, local):
         dist.barrier()
     torch.cuda.synchronize(dev)
     clocks.start()
-    time.sleep(0.3)  # let the sampler take its first reading
+    time.sleep(0.3)  # let the sampler take its first readings
+    wall0 = time.time()
     t0.record(stream)
     for i in range(args.steps):
         step(attn_events[i])
     t1.record(stream)
     torch.cuda.synchronize(dev)
-    clk = clocks.stop()
+    wall1 = time.time()
+    clk = clocks.stop(wall0, wall1)
     if dist is not None:
         dist.barrier()
     elapsed_ms = t0.elapsed_time(t1)

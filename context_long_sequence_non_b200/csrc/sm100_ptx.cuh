@@ -60,16 +60,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete yet is parked by
+// the hardware (up to `ns` nanoseconds, or until the phase completes) instead of spinning
+// and taking issue slots from the warps it shares a sub-partition with.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity.  Returns false when the CTA-wide
 // abort flag is already up or when `limit` SM cycles pass without completion; in the
 // latter case it raises the abort flag and records kDevErrTimeout in `err`.  No trap,
-// no unbounded spin: a stalled pipeline ends in an error status.
+// no unbounded spin: a stalled pipeline ends in an error status.  The clock and the
+// abort flag are checked every 64 parked tries (each parks for at most 20 us).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           int* err, long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if (*abort_flag) return false;
     if (clock64() - t0 > limit) {
       *abort_flag = 1;
@@ -86,6 +104,21 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, long l
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity) && clock64() - t0 < limit) {
   }
+}
+
+// Named-barrier rendezvous of `count` threads on barrier `id` that also ANDs a predicate
+// across them: every participant learns whether all of them passed `ok`.
+__device__ __forceinline__ bool bar_and(uint32_t id, uint32_t count, bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"(ok ? 1u : 0u), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
 }
 
 // ------------------------------------------------------------------ TMA
