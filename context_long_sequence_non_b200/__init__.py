@@ -16,6 +16,8 @@ from ._binding import (  # noqa: F401
     CpattnError,
     device_error,
     fwd,
+    fwd_accumulate,
+    ulysses_fwd,
     head2seq,
     lib,
     library_path,
@@ -23,6 +25,7 @@ from ._binding import (  # noqa: F401
     selftest_exp2,
     selftest_wait_timeout,
     seq2head,
+    seq2head_qkv,
     status_str,
     version,
 )

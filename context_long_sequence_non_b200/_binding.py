@@ -47,16 +47,19 @@ def lib() -> ctypes.CDLL:
             L = ctypes.CDLL(LIB_PATH)
             vp, i, f, ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong
             L.cpattn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+            L.cpattn_fwd_accumulate.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+            L.cpattn_ulysses_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
             L.cpattn_merge.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
             L.cpattn_seq2head.argtypes = [vp, vp, i, i, i, i, i, vp]
             L.cpattn_head2seq.argtypes = [vp, vp, i, i, i, i, i, vp]
+            L.cpattn_seq2head_qkv.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
             L.cpattn_status_str.argtypes = [i]
             L.cpattn_status_str.restype = ctypes.c_char_p
             L.cpattn_device_error.argtypes = []
             L.cpattn_selftest_wait_timeout.argtypes = [ll, vp]
             L.cpattn_version.argtypes = []
             L.cpattn_selftest_exp2.argtypes = [vp, vp, i, vp]
-            for name in ("cpattn_fwd", "cpattn_merge", "cpattn_seq2head", "cpattn_head2seq",
+            for name in ("cpattn_fwd", "cpattn_fwd_accumulate", "cpattn_ulysses_fwd", "cpattn_merge", "cpattn_seq2head_qkv", "cpattn_seq2head", "cpattn_head2seq",
                          "cpattn_device_error", "cpattn_selftest_wait_timeout", "cpattn_version",
                          "cpattn_selftest_exp2"):
                 getattr(L, name).restype = ctypes.c_int
@@ -126,6 +129,45 @@ def fwd(q, k, v, out=None, lse=None, scale=None, out_dtype=None, want_lse=True, 
     return out, lse
 
 
+def ulysses_fwd(q, k, v, P, out=None, lse=None, scale=None, out_dtype=None, want_lse=True,
+                stream=None):
+    """Ulysses attention in one kernel: q/k/v/out are [P][S_l][H][D] rank shards; returns
+    ``(out, lse [P][H/P][P*S_l])`` equal to seq2head -> fwd -> head2seq."""
+    P_, S_l, H, D = q.shape
+    if P_ != P or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must be same-shaped [P][S_l][H][D] shards")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty((P, S_l, H, D), dtype=out_dtype or q.dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((P, H // P, P * S_l), dtype=torch.float32, device=q.device)
+    _need_cuda(q, k, v, out, lse)
+    st = lib().cpattn_ulysses_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), P, S_l, H, D,
+                                  float(scale), _dtype_code(out.dtype), _stream(stream))
+    _check(st, "cpattn_ulysses_fwd")
+    return out, lse
+
+
+def fwd_accumulate(q, k, v, o_acc, lse_acc, scale=None, stream=None):
+    """Ring Attention step with the merge fused into the attention epilogue: attention of
+    q over this K/V chunk, merged in place into the running (o_acc, lse_acc)."""
+    B, Sq, H, D = q.shape
+    Skv = k.shape[1]
+    if k.shape != (B, Skv, H, D) or v.shape != (B, Skv, H, D):
+        raise ValueError("k and v must be [B][Skv][H][D] matching q")
+    if o_acc.shape != (B, Sq, H, D) or lse_acc.shape != (B, H, Sq):
+        raise ValueError("o_acc must be [B][Sq][H][D] and lse_acc [B][H][Sq]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    _need_cuda(q, k, v, o_acc, lse_acc)
+    st = lib().cpattn_fwd_accumulate(_ptr(q), _ptr(k), _ptr(v), _ptr(o_acc), _ptr(lse_acc), B, H,
+                                     Sq, Skv, D, float(scale), _dtype_code(q.dtype),
+                                     _dtype_code(o_acc.dtype), _stream(stream))
+    _check(st, "cpattn_fwd_accumulate")
+    return o_acc, lse_acc
+
+
 def merge(o_a, lse_a, o_b, lse_b, out=None, lse=None, stream=None):
     """Exact merge of two partial (O, LSE) results; ``out``/``lse`` may be o_a/lse_a."""
     B, S, H, D = o_a.shape
@@ -151,6 +193,21 @@ def seq2head(src, P, out=None, stream=None):
     st = lib().cpattn_seq2head(_ptr(src), _ptr(out), P, S_l, H, D, src.element_size(),
                                _stream(stream))
     _check(st, "cpattn_seq2head")
+    return out
+
+
+def seq2head_qkv(q, k, v, P, out=None, stream=None):
+    """seq2head of Q, K and V in one launch; ``out`` is an optional (qh, kh, vh) triple."""
+    P_, S_l, H, D = q.shape
+    if P_ != P or k.shape != q.shape or v.shape != q.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must be same-shaped [P][S_l][H][D] tensors")
+    if out is None:
+        out = tuple(torch.empty((P, P * S_l, H // P, D), dtype=q.dtype, device=q.device)
+                    for _ in range(3))
+    _need_cuda(q, k, v, *out)
+    st = lib().cpattn_seq2head_qkv(_ptr(q), _ptr(k), _ptr(v), *(_ptr(t) for t in out), P, S_l, H,
+                                   D, q.element_size(), _stream(stream))
+    _check(st, "cpattn_seq2head_qkv")
     return out
 
 

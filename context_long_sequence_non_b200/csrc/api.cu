@@ -46,15 +46,16 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [B][S][H][D] bf16 tensor, box = 64 head-dim columns x 1 head x 128 tokens x 1 batch,
-// 128-byte swizzle (the layout tcgen05 reads through a 128-byte-swizzle descriptor).
-bool encode_bshd_bf16(CUtensorMap* map, const void* ptr, int B, int S, int H, int D) {
+// [B][S][H][D] bf16 tensor, box = 64 head-dim columns x 1 head x `box_rows` tokens x 1
+// batch, 128-byte swizzle (the layout tcgen05 reads through a 128-byte-swizzle descriptor).
+bool encode_bshd_bf16(CUtensorMap* map, const void* ptr, int B, int S, int H, int D,
+                      unsigned box_rows = 128) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(S), cuuint64_t(B)};
   const cuuint64_t strides[3] = {cuuint64_t(D) * 2, cuuint64_t(H) * D * 2,
                                  cuuint64_t(S) * H * D * 2};
-  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t box[4] = {64, 1, box_rows, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -94,14 +95,20 @@ const char* cpattn_status_str(int status) {
   }
 }
 
-int cpattn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
-               int Sq, int Skv, int D, float scale, int in_dtype, int out_dtype,
-               cpattn_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+int fwd_impl(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
+             int Sq, int Skv, int D, float scale, int in_dtype, int out_dtype, bool accumulate,
+             cpattn_stream_t stream) {
   if (B < 1 || H < 1 || Sq < 1 || Skv < 0 || D < 1) return CPATTN_ERR_SHAPE;
   if (!(std::isfinite(scale) && scale > 0.f)) return CPATTN_ERR_SHAPE;
   const int in_es = elem_size(in_dtype), out_es = elem_size(out_dtype);
   if (in_es == 0 || out_es == 0) return CPATTN_ERR_UNSUPPORTED;
+  if (accumulate && in_dtype != CPATTN_BF16) return CPATTN_ERR_UNSUPPORTED;
   if (q == nullptr || out == nullptr) return CPATTN_ERR_NULL;
+  if (accumulate && lse == nullptr) return CPATTN_ERR_NULL;
   if (Skv > 0 && (k == nullptr || v == nullptr)) return CPATTN_ERR_NULL;
   if (!aligned(q, 16) || !aligned(out, 16) || (Skv > 0 && (!aligned(k, 16) || !aligned(v, 16))) ||
       (lse != nullptr && !aligned(lse, 4)))
@@ -112,6 +119,7 @@ int cpattn_fwd(const void* q, const void* k, const void* v, void* out, float* ls
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const size_t out_bytes = size_t(B) * Sq * H * D * out_es;
   if (Skv == 0) {
+    if (accumulate) return CPATTN_OK;  // merging an empty key set changes nothing
     if (out_bytes % 16 != 0) return CPATTN_ERR_SHAPE;
     return cuda_status(cpattn::launch_fill_empty(out, out_bytes, lse, size_t(B) * H * Sq, st));
   }
@@ -125,12 +133,57 @@ int cpattn_fwd(const void* q, const void* k, const void* v, void* out, float* ls
     const float scale_log2 = float(double(scale) * 1.4426950408889634074);
     return cuda_status(cpattn::launch_attn_fwd_sm100(
         tq, tk, tv, out, lse, B, H, Sq, Skv, D, scale_log2, cpattn::kRescaleLog2,
-        out_dtype == CPATTN_F32, err, cpattn::kDefaultWaitLimit, st));
+        out_dtype == CPATTN_F32, accumulate, err, cpattn::kDefaultWaitLimit, st));
   }
   // fp32 inputs: CUDA-core kernel
   return cuda_status(cpattn::launch_attn_fwd_f32(
       static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
       out, lse, B, H, Sq, Skv, D, scale, out_dtype == CPATTN_BF16, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+int cpattn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
+               int Sq, int Skv, int D, float scale, int in_dtype, int out_dtype,
+               cpattn_stream_t stream) {
+  return fwd_impl(q, k, v, out, lse, B, H, Sq, Skv, D, scale, in_dtype, out_dtype, false, stream);
+}
+
+int cpattn_fwd_accumulate(const void* q, const void* k, const void* v, void* o_acc,
+                          float* lse_acc, int B, int H, int Sq, int Skv, int D, float scale,
+                          int in_dtype, int acc_dtype, cpattn_stream_t stream) {
+  return fwd_impl(q, k, v, o_acc, lse_acc, B, H, Sq, Skv, D, scale, in_dtype, acc_dtype, true,
+                  stream);
+}
+
+int cpattn_ulysses_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int P,
+                       int S_local, int H, int D, float scale, int out_dtype,
+                       cpattn_stream_t stream) {
+  if (P < 1 || S_local < 1 || H < 1 || D < 1) return CPATTN_ERR_SHAPE;
+  if (H % P != 0) return CPATTN_ERR_SHAPE;
+  if ((long long)P * S_local > 0x7fffffffLL || P > 65535 || H / P > 65535) return CPATTN_ERR_SHAPE;
+  if (!(std::isfinite(scale) && scale > 0.f)) return CPATTN_ERR_SHAPE;
+  if (elem_size(out_dtype) == 0) return CPATTN_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return CPATTN_ERR_UNSUPPORTED;
+  if (S_local % 16 != 0) return CPATTN_ERR_UNSUPPORTED;  // 16-row boxes may not cross shards
+  if (!q || !k || !v || !out) return CPATTN_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      (lse != nullptr && !aligned(lse, 4)))
+    return CPATTN_ERR_ALIGN;
+  int* err = device_error_word();
+  if (err == nullptr) return CPATTN_ERR_CUDA;
+  CUtensorMap tq, tk, tv;
+  if (!encode_bshd_bf16(&tq, q, P, S_local, H, D, 16) ||
+      !encode_bshd_bf16(&tk, k, P, S_local, H, D, 16) ||
+      !encode_bshd_bf16(&tv, v, P, S_local, H, D, 16))
+    return CPATTN_ERR_CUDA;
+  const float scale_log2 = float(double(scale) * 1.4426950408889634074);
+  return cuda_status(cpattn::launch_ulysses_fwd_sm100(
+      tq, tk, tv, out, lse, P, S_local, H, D, scale_log2, cpattn::kRescaleLog2,
+      out_dtype == CPATTN_F32, err, cpattn::kDefaultWaitLimit,
+      reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int cpattn_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b, void* o,
@@ -176,6 +229,25 @@ int cpattn_seq2head(const void* src, void* dst, int P, int S_local, int H, int D
   if (st != CPATTN_OK) return st;
   return cuda_status(cpattn::launch_seq2head(src, dst, P, S_local, run_vec,
                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int cpattn_seq2head_qkv(const void* q, const void* k, const void* v, void* qh, void* kh, void* vh,
+                        int P, int S_local, int H, int D, int elem_bytes, cpattn_stream_t stream) {
+  const void* src[3] = {q, k, v};
+  void* dst[3] = {qh, kh, vh};
+  long long run_vec = 0;
+  for (int t = 0; t < 3; ++t) {
+    const int st = permute_args(src[t], dst[t], P, S_local, H, D, elem_bytes, &run_vec);
+    if (st != CPATTN_OK) return st;
+  }
+  // no destination may overlap another tensor's source or destination
+  const size_t bytes = size_t(P) * S_local * H * D * elem_bytes;
+  for (int a = 0; a < 3; ++a)
+    for (int c = 0; c < 3; ++c)
+      if ((a != c && overlap(dst[a], bytes, dst[c], bytes)) || overlap(dst[a], bytes, src[c], bytes))
+        return CPATTN_ERR_SHAPE;
+  return cuda_status(cpattn::launch_seq2head_n(src, dst, 3, P, S_local, run_vec,
+                                               reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int cpattn_head2seq(const void* src, void* dst, int P, int S_local, int H, int D, int elem_bytes,

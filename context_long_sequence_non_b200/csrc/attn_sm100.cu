@@ -44,6 +44,8 @@ constexpr uint32_t kRegsLaunch = 168, kRegsSoftmax = 216, kRegsOther = 72;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kRegsLaunch * kThreads,
               "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
+constexpr float kLn2 = 0.69314718055994530942f;
+constexpr float kLog2e = 1.44269504088896340736f;
 // exp2 work split: of every 8 column pairs, this many go through the FMA-pipe polynomial
 // and the rest through the special-function unit (ex2), which would otherwise be
 // co-critical with the tensor core (one ex2 per score, 16 per clock per SM).
@@ -73,14 +75,29 @@ struct __align__(8) Barriers {
   uint64_t drain;
 };
 
-template <int D, bool kOutF32>
+// Addressing/epilogue modes of the kernel.
+enum Mode : int {
+  kPlain = 0,    // [B][S][H][D] in, O and LSE written
+  kAccum = 1,    // as kPlain, but (O, LSE) merged into the running accumulator in place
+  kSharded = 2,  // Ulysses fused: Q/K/V/O are [P][S_l][H*P][D] rank shards (see below)
+};
+
+template <int D, bool kOutF32, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, void* __restrict__ out,
                           float* __restrict__ lse, int H, int Sq, int Skv, float scale_log2,
-                          float rescale_log2, int* err, long long wait_limit) {
+                          float rescale_log2, int s_local, int* err, long long wait_limit) {
   using G = Geometry<D>;
+  constexpr bool kAcc = kMode == kAccum;
+  // kSharded: the DeepSpeed Ulysses path in one kernel.  The grid's z is the head group g
+  // (P of them), y the head j inside it (H = heads per group); head g*H + j of the full
+  // sequence is read straight from the sequence shards [P][S_l][H*P][D] (token t lives in
+  // shard t / S_l, row t % S_l) with 16-row TMA boxes, so no box crosses a shard boundary
+  // (S_l % 16 == 0), and O goes back to the same sharded layout: the all-to-alls become
+  // addressing.
+  constexpr bool kShard = kMode == kSharded;
   extern __shared__ uint8_t smem_raw[];
   __shared__ Barriers bars;
   __shared__ uint32_t tmem_base_sh;
@@ -94,6 +111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int q_first = blockIdx.x * (2 * kBlockM);
   const int h = blockIdx.y;
   const int b = blockIdx.z;
+  const int head_coord = kShard ? b * H + h : h;  // head coordinate in the tensor maps
   const int n_kv = (Skv + kBlockN - 1) / kBlockN;
   volatile int* abort_flag = &abort_sh;
 
@@ -253,8 +271,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int q = q_first + tile * kBlockM + row;
       const bool in_range = q < Sq;
-      const float inv_l = 1.0f / l;
-      const size_t row_off = ((size_t(b) * Sq + (in_range ? q : 0)) * H + h) * size_t(D);
+      const int qr = in_range ? q : 0;
+      // sharded layout: token q = r * S_l + s sits at row q of the flattened [P][S_l] shards
+      const size_t row_off = kShard ? (size_t(qr) * (H * gridDim.z) + head_coord) * size_t(D)
+                                    : ((size_t(b) * Sq + qr) * H + h) * size_t(D);
+      const size_t lse_idx = (size_t(b) * H + h) * Sq + (in_range ? q : 0);
+      // this block's result: O_c = O_tmem / l, LSE_c = ln(2^m * l) = (m + log2 l) * ln 2
+      const float lc2 = m + log2f(l);  // LSE_c in base 2
+      float fa = 0.f, fc = 1.0f / l;   // written row = fa * O_acc + fc * O_tmem
+      float lse_out = lc2 * kLn2;
+      if constexpr (kAcc) {
+        // Ring Attention step fused into the epilogue: merge (O_c, LSE_c) into the running
+        // (O_acc, LSE_acc) in place; an empty accumulator (LSE_acc = -inf) takes O_c
+        if (in_range) {
+          const float la2 = lse[lse_idx] * kLog2e;
+          const float mx = fmaxf(la2, lc2);
+          const float wa = exp2f(la2 - mx), wc = exp2f(lc2 - mx);
+          const float tot = wa + wc;
+          fa = wa / tot;
+          fc = wc / (tot * l);
+          lse_out = (mx + log2f(tot)) * kLn2;
+        }
+      }
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
@@ -263,29 +301,45 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (kOutF32) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + row_off + c * 32);
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              dst[e] = make_float4(__uint_as_float(r[4 * e]) * inv_l,
-                                   __uint_as_float(r[4 * e + 1]) * inv_l,
-                                   __uint_as_float(r[4 * e + 2]) * inv_l,
-                                   __uint_as_float(r[4 * e + 3]) * inv_l);
+            for (int e = 0; e < 8; ++e) {
+              float4 v = make_float4(__uint_as_float(r[4 * e]) * fc, __uint_as_float(r[4 * e + 1]) * fc,
+                                     __uint_as_float(r[4 * e + 2]) * fc, __uint_as_float(r[4 * e + 3]) * fc);
+              if (kAcc && fa != 0.f) {  // an empty accumulator row is never read
+                const float4 a = dst[e];
+                v.x = fmaf(fa, a.x, v.x);
+                v.y = fmaf(fa, a.y, v.y);
+                v.z = fmaf(fa, a.z, v.z);
+                v.w = fmaf(fa, a.w, v.w);
+              }
+              dst[e] = v;
+            }
           } else {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + row_off + c * 32);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
+              float o[8];
+#pragma unroll
+              for (int t = 0; t < 8; ++t) o[t] = __uint_as_float(r[8 * e + t]) * fc;
+              if (kAcc && fa != 0.f) {  // an empty accumulator row is never read
+                const uint4 a = dst[e];
+                const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                  o[2 * t] = fmaf(fa, __uint_as_float(aw[t] << 16), o[2 * t]);
+                  o[2 * t + 1] = fmaf(fa, __uint_as_float(aw[t] & 0xFFFF0000u), o[2 * t + 1]);
+                }
+              }
               uint4 v;
-              v.x = pack_bf16x2(__uint_as_float(r[8 * e + 0]) * inv_l, __uint_as_float(r[8 * e + 1]) * inv_l);
-              v.y = pack_bf16x2(__uint_as_float(r[8 * e + 2]) * inv_l, __uint_as_float(r[8 * e + 3]) * inv_l);
-              v.z = pack_bf16x2(__uint_as_float(r[8 * e + 4]) * inv_l, __uint_as_float(r[8 * e + 5]) * inv_l);
-              v.w = pack_bf16x2(__uint_as_float(r[8 * e + 6]) * inv_l, __uint_as_float(r[8 * e + 7]) * inv_l);
+              v.x = pack_bf16x2(o[0], o[1]);
+              v.y = pack_bf16x2(o[2], o[3]);
+              v.z = pack_bf16x2(o[4], o[5]);
+              v.w = pack_bf16x2(o[6], o[7]);
               dst[e] = v;
             }
           }
         }
       }
-      if (in_range && lse != nullptr) {
-        // LSE = ln(2^m * l) = (m + log2 l) * ln 2
-        lse[(size_t(b) * H + h) * Sq + q] = (m + log2f(l)) * 0.69314718055994530942f;
-      }
+      if (in_range && lse != nullptr) lse[lse_idx] = lse_out;
     }
   } else {
     regs_dec<kRegsOther>();
@@ -293,14 +347,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kWarpProducer) {
     // ------------------------------------------------------------------ TMA producer
     if (elect_one()) {
+      // one 128-row tile starting at token t0 into `dst`: a 64-column box per 128-byte
+      // column block; sharded inputs take eight 16-row boxes, each inside one rank shard
+      auto load_tile = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, int t0) {
+#pragma unroll
+        for (int bx = 0; bx < G::kBoxes; ++bx) {
+          if constexpr (!kShard) {
+            tma_load_4d(dst + bx * G::kBoxBytes, map, bar, bx * G::kBox, head_coord, t0, b);
+          } else {
+#pragma unroll 1
+            for (int i = 0; i < kBlockN / 16; ++i) {
+              const int t = t0 + 16 * i;
+              const int r = t / s_local;  // rank shard (== P past the end: zero-filled)
+              tma_load_4d(dst + bx * G::kBoxBytes + i * 16 * 128, map, bar, bx * G::kBox,
+                          head_coord, t - r * s_local, r);
+            }
+          }
+        }
+      };
       const uint32_t bar_q = smem_u32(&bars.q_full);
       mbar_arrive_expect_tx(bar_q, 2 * G::kTileBytes);
 #pragma unroll
       for (int t = 0; t < 2; ++t)
-#pragma unroll
-        for (int bx = 0; bx < G::kBoxes; ++bx)
-          tma_load_4d(smem_base + G::kOffQ + t * G::kTileBytes + bx * G::kBoxBytes, &tm_q, bar_q,
-                      bx * G::kBox, h, q_first + t * kBlockM, b);
+        load_tile(&tm_q, smem_base + G::kOffQ + t * G::kTileBytes, bar_q, q_first + t * kBlockM);
       int issued = 0;
       for (int use = 0; use < 2 * n_kv; ++use) {
         const int slot = use % kSlots;
@@ -309,11 +378,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t bar_f = smem_u32(&bars.full[slot]);
         mbar_arrive_expect_tx(bar_f, G::kTileBytes);
         const CUtensorMap* map = (use & 1) ? &tm_v : &tm_k;
-        const int key0 = (use >> 1) * kBlockN;
-#pragma unroll
-        for (int bx = 0; bx < G::kBoxes; ++bx)
-          tma_load_4d(smem_base + G::kOffSlots + slot * G::kTileBytes + bx * G::kBoxBytes, map,
-                      bar_f, bx * G::kBox, h, key0, b);
+        load_tile(map, smem_base + G::kOffSlots + slot * G::kTileBytes, bar_f,
+                  (use >> 1) * kBlockN);
         issued = use + 1;
       }
       // drain: every issued copy must have landed before the CTA's shared memory is
@@ -405,19 +471,59 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kWarpMma) tmem_dealloc(tmem, kTmemCols);
 }
 
-template <int D, bool kOutF32>
+template <int D, bool kOutF32, int kMode>
 cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* out,
-                   float* lse, int B, int H, int Sq, int Skv, float scale_log2,
-                   float rescale_log2, int* err, long long wait_limit, cudaStream_t stream) {
+                   float* lse, dim3 grid, int H, int Sq, int Skv, float scale_log2,
+                   float rescale_log2, int s_local, int* err, long long wait_limit,
+                   cudaStream_t stream) {
   using G = Geometry<D>;
-  auto kernel = attn_fwd_sm100_kernel<D, kOutF32>;
+  auto kernel = attn_fwd_sm100_kernel<D, kOutF32, kMode>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        G::kDynSmem);
   if (e != cudaSuccess) return e;
-  dim3 grid((Sq + 2 * kBlockM - 1) / (2 * kBlockM), H, B);
   kernel<<<grid, kThreads, G::kDynSmem, stream>>>(tq, tk, tv, out, lse, H, Sq, Skv, scale_log2,
-                                                   rescale_log2, err, wait_limit);
+                                                   rescale_log2, s_local, err, wait_limit);
   return cudaGetLastError();
+}
+
+template <int D, int kMode>
+cudaError_t launch_o(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* out,
+                     float* lse, dim3 grid, int H, int Sq, int Skv, float scale_log2,
+                     float rescale_log2, int s_local, bool out_f32, int* err, long long wait_limit,
+                     cudaStream_t stream) {
+  return out_f32 ? launch<D, true, kMode>(tq, tk, tv, out, lse, grid, H, Sq, Skv, scale_log2,
+                                          rescale_log2, s_local, err, wait_limit, stream)
+                 : launch<D, false, kMode>(tq, tk, tv, out, lse, grid, H, Sq, Skv, scale_log2,
+                                           rescale_log2, s_local, err, wait_limit, stream);
+}
+
+template <int D>
+cudaError_t launch_m(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* out,
+                     float* lse, dim3 grid, int H, int Sq, int Skv, float scale_log2,
+                     float rescale_log2, int s_local, bool out_f32, int mode, int* err,
+                     long long wait_limit, cudaStream_t stream) {
+  switch (mode) {
+    case kAccum:
+      return launch_o<D, kAccum>(tq, tk, tv, out, lse, grid, H, Sq, Skv, scale_log2, rescale_log2,
+                                 s_local, out_f32, err, wait_limit, stream);
+    case kSharded:
+      return launch_o<D, kSharded>(tq, tk, tv, out, lse, grid, H, Sq, Skv, scale_log2,
+                                   rescale_log2, s_local, out_f32, err, wait_limit, stream);
+    default:
+      return launch_o<D, kPlain>(tq, tk, tv, out, lse, grid, H, Sq, Skv, scale_log2, rescale_log2,
+                                 s_local, out_f32, err, wait_limit, stream);
+  }
+}
+
+cudaError_t launch_any(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       void* out, float* lse, dim3 grid, int H, int Sq, int Skv, int D,
+                       float scale_log2, float rescale_log2, int s_local, bool out_f32, int mode,
+                       int* err, long long wait_limit, cudaStream_t stream) {
+  if (D == 128)
+    return launch_m<128>(tq, tk, tv, out, lse, grid, H, Sq, Skv, scale_log2, rescale_log2, s_local,
+                         out_f32, mode, err, wait_limit, stream);
+  return launch_m<64>(tq, tk, tv, out, lse, grid, H, Sq, Skv, scale_log2, rescale_log2, s_local,
+                      out_f32, mode, err, wait_limit, stream);
 }
 
 }  // namespace
@@ -425,18 +531,22 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
 cudaError_t launch_attn_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
                                   const CUtensorMap& tv, void* out, float* lse, int B, int H,
                                   int Sq, int Skv, int D, float scale_log2, float rescale_log2,
-                                  bool out_f32, int* err, long long wait_limit,
+                                  bool out_f32, bool accumulate, int* err, long long wait_limit,
                                   cudaStream_t stream) {
-  if (D == 128) {
-    return out_f32 ? launch<128, true>(tq, tk, tv, out, lse, B, H, Sq, Skv, scale_log2,
-                                       rescale_log2, err, wait_limit, stream)
-                   : launch<128, false>(tq, tk, tv, out, lse, B, H, Sq, Skv, scale_log2,
-                                        rescale_log2, err, wait_limit, stream);
-  }
-  return out_f32 ? launch<64, true>(tq, tk, tv, out, lse, B, H, Sq, Skv, scale_log2,
-                                    rescale_log2, err, wait_limit, stream)
-                 : launch<64, false>(tq, tk, tv, out, lse, B, H, Sq, Skv, scale_log2,
-                                     rescale_log2, err, wait_limit, stream);
+  const dim3 grid((Sq + 2 * kBlockM - 1) / (2 * kBlockM), H, B);
+  return launch_any(tq, tk, tv, out, lse, grid, H, Sq, Skv, D, scale_log2, rescale_log2, 0,
+                    out_f32, accumulate ? kAccum : kPlain, err, wait_limit, stream);
+}
+
+cudaError_t launch_ulysses_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
+                                     const CUtensorMap& tv, void* out, float* lse, int P,
+                                     int S_local, int H, int D, float scale_log2,
+                                     float rescale_log2, bool out_f32, int* err,
+                                     long long wait_limit, cudaStream_t stream) {
+  const int S = P * S_local, Hp = H / P;
+  const dim3 grid((S + 2 * kBlockM - 1) / (2 * kBlockM), Hp, P);
+  return launch_any(tq, tk, tv, out, lse, grid, Hp, S, S, D, scale_log2, rescale_log2, S_local,
+                    out_f32, kSharded, err, wait_limit, stream);
 }
 
 }  // namespace cpattn

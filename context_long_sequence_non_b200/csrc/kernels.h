@@ -11,12 +11,21 @@ namespace cpattn {
 constexpr long long kDefaultWaitLimit = 2000000000LL;
 
 // tcgen05 attention, bf16 in, D in {64, 128}; tensor maps describe [B][S][H][D] bf16
-// tensors with a 64 x 1 x 128 x 1 box and 128-byte swizzle.
+// tensors with a 64 x 1 x 128 x 1 box and 128-byte swizzle.  With `accumulate` the result
+// is merged into (out, lse) in place (the Ring Attention step) instead of overwriting it.
 cudaError_t launch_attn_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
                                   const CUtensorMap& tv, void* out, float* lse, int B, int H,
                                   int Sq, int Skv, int D, float scale_log2, float rescale_log2,
-                                  bool out_f32, int* err, long long wait_limit,
+                                  bool out_f32, bool accumulate, int* err, long long wait_limit,
                                   cudaStream_t stream);
+
+// Ulysses fused: q/k/v/out are [P][S_local][H][D] rank shards (tensor maps with a
+// 64 x 1 x 16 x 1 box over dims (D, H, S_local, P)); LSE is [P][H/P][P*S_local].
+cudaError_t launch_ulysses_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
+                                     const CUtensorMap& tv, void* out, float* lse, int P,
+                                     int S_local, int H, int D, float scale_log2,
+                                     float rescale_log2, bool out_f32, int* err,
+                                     long long wait_limit, cudaStream_t stream);
 
 // Running-max policy of the tensor-core kernel: 0 = exact running max (the dominant key's
 // P is exactly 1, so its bf16 rounding costs nothing).
@@ -41,6 +50,9 @@ cudaError_t launch_seq2head(const void* src, void* dst, int P, int S_local, long
                             cudaStream_t stream);
 cudaError_t launch_head2seq(const void* src, void* dst, int P, int S_local, long long run_vec,
                             cudaStream_t stream);
+// seq2head of n (1..3) same-shaped tensors in one launch.
+cudaError_t launch_seq2head_n(const void* const* src, void* const* dst, int n, int P, int S_local,
+                              long long run_vec, cudaStream_t stream);
 
 // One CTA waiting on an mbarrier nothing completes, with the attention kernel's bounded wait.
 cudaError_t launch_wait_timeout_selftest(int* err, long long limit, cudaStream_t stream);

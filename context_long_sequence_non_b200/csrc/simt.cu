@@ -168,24 +168,33 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
 constexpr int kPermThreads = 256;
 constexpr int kPermUnroll = 4;
 
+// Up to three tensors share one launch (Q, K and V go through the same re-partition).
+struct PermuteSet {
+  const uint4* src[3];
+  uint4* dst[3];
+};
+
 template <bool kToHead>
-__global__ void __launch_bounds__(kPermThreads) permute_kernel(const uint4* __restrict__ src,
-                                                                uint4* __restrict__ dst, int P,
-                                                                int S_l, int run_vec, int chunks,
+__global__ void __launch_bounds__(kPermThreads) permute_kernel(const __grid_constant__ PermuteSet set,
+                                                                int n_tensors, int P, int S_l,
+                                                                int run_vec, int chunks,
                                                                 long long n_items) {
   const int lane = threadIdx.x & 31;
   const long long warp = ((long long)blockIdx.x * kPermThreads + threadIdx.x) >> 5;
   const long long n_warps = ((long long)gridDim.x * kPermThreads) >> 5;
-  for (long long it0 = warp * kPermUnroll; it0 < n_items; it0 += n_warps * kPermUnroll) {
+  const long long total = n_items * n_tensors;
+  for (long long it0 = warp * kPermUnroll; it0 < total; it0 += n_warps * kPermUnroll) {
     uint4 buf[kPermUnroll];
-    long long dst_off[kPermUnroll];
+    uint4* dst_ptr[kPermUnroll];
     bool live[kPermUnroll];
 #pragma unroll
     for (int u = 0; u < kPermUnroll; ++u) {
-      const long long it = it0 + u;
+      const long long itg = it0 + u;
+      const int tsel = int(itg / n_items);  // which tensor
+      const long long it = itg - (long long)tsel * n_items;
       const long long n = it / chunks;  // dst row
       const int v = int(it - n * chunks) * 32 + lane;
-      live[u] = it < n_items && v < run_vec;
+      live[u] = itg < total && v < run_vec;
       long long src_row = 0;
       if (kToHead) {  // n = A(g, r, s)
         const int s = int(n % S_l);
@@ -200,12 +209,13 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const uint4* __re
         const int r = int(rs / S_l);
         src_row = ((long long)g * P + r) * S_l + s;
       }
-      dst_off[u] = n * run_vec + v;
-      if (live[u]) buf[u] = src[src_row * run_vec + v];
+      const int ts = live[u] ? tsel : 0;
+      dst_ptr[u] = set.dst[ts] + n * run_vec + v;
+      if (live[u]) buf[u] = set.src[ts][src_row * run_vec + v];
     }
 #pragma unroll
     for (int u = 0; u < kPermUnroll; ++u)
-      if (live[u]) dst[dst_off[u]] = buf[u];
+      if (live[u]) *dst_ptr[u] = buf[u];
   }
 }
 
@@ -317,34 +327,48 @@ cudaError_t launch_merge(const void* o_a, const float* lse_a, const void* o_b, c
   return cudaGetLastError();
 }
 
-static cudaError_t launch_permute(bool to_head, const void* src, void* dst, int P, int S_local,
-                                  long long run_vec, cudaStream_t stream) {
+static cudaError_t launch_permute(bool to_head, const void* const* src, void* const* dst,
+                                  int n_tensors, int P, int S_local, long long run_vec,
+                                  cudaStream_t stream) {
+  PermuteSet set{};
+  for (int t = 0; t < 3; ++t) {
+    const int u = t < n_tensors ? t : 0;
+    set.src[t] = static_cast<const uint4*>(src[u]);
+    set.dst[t] = static_cast<uint4*>(dst[u]);
+  }
   const long long n_rows = (long long)P * P * S_local;
   const int chunks = int((run_vec + 31) / 32);
   const long long n_items = n_rows * chunks;
-  const long long warps_needed = (n_items + kPermUnroll - 1) / kPermUnroll;
+  const long long warps_needed = (n_items * n_tensors + kPermUnroll - 1) / kPermUnroll;
   const long long blocks_needed = (warps_needed * 32 + kPermThreads - 1) / kPermThreads;
   const long long cap = (long long)sm_count() * 8;
   const long long blocks = blocks_needed < cap ? blocks_needed : cap;
   if (to_head)
     permute_kernel<true><<<unsigned(blocks), kPermThreads, 0, stream>>>(
-        static_cast<const uint4*>(src), static_cast<uint4*>(dst), P, S_local, int(run_vec), chunks,
-        n_items);
+        set, n_tensors, P, S_local, int(run_vec), chunks, n_items);
   else
     permute_kernel<false><<<unsigned(blocks), kPermThreads, 0, stream>>>(
-        static_cast<const uint4*>(src), static_cast<uint4*>(dst), P, S_local, int(run_vec), chunks,
-        n_items);
+        set, n_tensors, P, S_local, int(run_vec), chunks, n_items);
   return cudaGetLastError();
 }
 
 cudaError_t launch_seq2head(const void* src, void* dst, int P, int S_local, long long run_vec,
                             cudaStream_t stream) {
-  return launch_permute(true, src, dst, P, S_local, run_vec, stream);
+  const void* s[1] = {src};
+  void* d[1] = {dst};
+  return launch_permute(true, s, d, 1, P, S_local, run_vec, stream);
 }
 
 cudaError_t launch_head2seq(const void* src, void* dst, int P, int S_local, long long run_vec,
                             cudaStream_t stream) {
-  return launch_permute(false, src, dst, P, S_local, run_vec, stream);
+  const void* s[1] = {src};
+  void* d[1] = {dst};
+  return launch_permute(false, s, d, 1, P, S_local, run_vec, stream);
+}
+
+cudaError_t launch_seq2head_n(const void* const* src, void* const* dst, int n, int P, int S_local,
+                              long long run_vec, cudaStream_t stream) {
+  return launch_permute(true, src, dst, n, P, S_local, run_vec, stream);
 }
 
 cudaError_t launch_exp2_poly_selftest(const float* t, float* out, int n, cudaStream_t stream) {

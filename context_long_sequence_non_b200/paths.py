@@ -19,12 +19,14 @@ import torch
 from . import _binding as B
 
 
-def ring_attention(q, k_chunks, v_chunks, scale=None, acc_dtype=None, stream=None):
+def ring_attention(q, k_chunks, v_chunks, scale=None, acc_dtype=None, fused=True, stream=None):
     """One rank's ring step over K/V chunks in ring order.
 
     q: [B][Sq][H][D]; each chunk [B][S_c][H][D].  The running (O, LSE) is kept in
-    ``acc_dtype`` (default: q's dtype); chunk partials are produced in the same dtype and
-    merged in place.  Returns ``(O, LSE)``.
+    ``acc_dtype`` (default: q's dtype).  ``fused=True`` (default) merges every chunk into
+    the accumulator inside the attention epilogue (cpattn_fwd_accumulate); ``fused=False``
+    writes each chunk's partial and folds it with the separate merge kernel.  Returns
+    ``(O, LSE)``.
     """
     if scale is None:
         scale = 1.0 / math.sqrt(q.shape[3])
@@ -32,6 +34,13 @@ def ring_attention(q, k_chunks, v_chunks, scale=None, acc_dtype=None, stream=Non
     Bn, Sq, H, D = q.shape
     acc_o = torch.empty((Bn, Sq, H, D), dtype=acc_dtype, device=q.device)
     acc_l = torch.empty((Bn, H, Sq), dtype=torch.float32, device=q.device)
+    if fused:
+        for c, (kc, vc) in enumerate(zip(k_chunks, v_chunks)):
+            if c == 0:
+                B.fwd(q, kc, vc, out=acc_o, lse=acc_l, scale=scale, stream=stream)
+            else:
+                B.fwd_accumulate(q, kc, vc, acc_o, acc_l, scale=scale, stream=stream)
+        return acc_o, acc_l
     tmp_o = torch.empty_like(acc_o)
     tmp_l = torch.empty_like(acc_l)
     for c, (kc, vc) in enumerate(zip(k_chunks, v_chunks)):
@@ -49,7 +58,8 @@ class UlyssesPlan:
     Shards are [P][S_l][H][D]; head-grouped buffers [P][P*S_l][H/P][D].
     """
 
-    def __init__(self, P, S_local, H, D, dtype=torch.bfloat16, device="cuda"):
+    def __init__(self, P, S_local, H, D, dtype=torch.bfloat16, device="cuda", batched=False):
+        self.batched = batched  # one seq2head launch for Q, K, V together
         if H % P:
             raise ValueError("H must be divisible by P")
         self.P, self.S_local, self.H, self.D = P, S_local, H, D
@@ -63,9 +73,13 @@ class UlyssesPlan:
 
     def run(self, q_shards, k_shards, v_shards, scale=None, stream=None):
         P = self.P
-        B.seq2head(q_shards, P, out=self.qh, stream=stream)
-        B.seq2head(k_shards, P, out=self.kh, stream=stream)
-        B.seq2head(v_shards, P, out=self.vh, stream=stream)
+        if self.batched:
+            B.seq2head_qkv(q_shards, k_shards, v_shards, P, out=(self.qh, self.kh, self.vh),
+                           stream=stream)
+        else:
+            B.seq2head(q_shards, P, out=self.qh, stream=stream)
+            B.seq2head(k_shards, P, out=self.kh, stream=stream)
+            B.seq2head(v_shards, P, out=self.vh, stream=stream)
         B.fwd(self.qh, self.kh, self.vh, out=self.oh, lse=self.lse, scale=scale, stream=stream)
         B.head2seq(self.oh, P, out=self.out, stream=stream)
         return self.out, self.lse

@@ -87,6 +87,46 @@ CPATTN_API int cpattn_fwd(const void* q, const void* k, const void* v, void* out
                int in_dtype, int out_dtype, cpattn_stream_t stream);
 
 /*
+ * cpattn_ulysses_fwd -- the whole DeepSpeed Ulysses attention of one layer in one kernel
+ * (Fig. 4: all-to-all from sequence shards to head groups, full-sequence attention per head
+ * group, all-to-all back), for P virtual ranks on one GPU.  The result equals
+ *   cpattn_seq2head (Q, K, V) -> cpattn_fwd (B = P, H = H/P, S = P*S_local) -> cpattn_head2seq
+ * but the re-partitions are done by the kernel's own addressing: every head is read over
+ * the full sequence straight from the rank shards and O is written back to them.
+ * q, k, v, out : [P][S_local][H][D] (q, k, v bf16; out BF16 or F32 per out_dtype).
+ * lse : [P][H/P][P*S_local] float32 (head group, head within group, token), or NULL.
+ * Requires H % P == 0, D in {64, 128}, S_local % 16 == 0 (the kernel reads 16-row boxes
+ * that must not straddle two shards; CPATTN_ERR_UNSUPPORTED otherwise), 0 < scale.
+ * Errors: CPATTN_ERR_NULL, _SHAPE, _ALIGN, _UNSUPPORTED, _CUDA.
+ */
+CPATTN_API int cpattn_ulysses_fwd(const void* q, const void* k, const void* v, void* out,
+                                  float* lse, int P, int S_local, int H, int D, float scale,
+                                  int out_dtype, cpattn_stream_t stream);
+
+/*
+ * cpattn_fwd_accumulate -- one Ring Attention step with the merge fused into the attention
+ * epilogue (环形注意力 / Ring Attention, Fig. 3: each rank folds every arriving K/V chunk
+ * into its running result with the online softmax).  Computes the chunk's partial
+ * (O_c, LSE_c) exactly as cpattn_fwd does and, instead of writing it out, merges it into
+ * the running accumulator in place:
+ *   L = max(L_acc, L_c) + ln(exp(L_acc - max) + exp(L_c - max))
+ *   O_acc = exp(L_acc - L) * O_acc + exp(L_c - L) * O_c,   L_acc = L
+ * Each accumulator row is read and rewritten by one thread, after the chunk is done.  A
+ * row with L_acc = -inf is an empty accumulator: its o_acc row is not read (it may hold
+ * anything, NaN included) and receives (O_c, L_c), so a ring step may start from an
+ * uninitialised o_acc with lse_acc = -inf.
+ * q : [B][Sq][H][D] bf16; k, v : [B][Skv][H][D] bf16 (the chunk); D in {64, 128}.
+ * o_acc : [B][Sq][H][D] in acc_dtype (BF16 or F32), lse_acc : [B][H][Sq] float32, both
+ * read and written.  Skv = 0 leaves the accumulator unchanged (nothing is launched).
+ * Errors: CPATTN_ERR_NULL (lse_acc is required), _SHAPE, _ALIGN, _UNSUPPORTED (in_dtype
+ * other than BF16, or D), _CUDA.
+ */
+CPATTN_API int cpattn_fwd_accumulate(const void* q, const void* k, const void* v, void* o_acc,
+                                     float* lse_acc, int B, int H, int Sq, int Skv, int D,
+                                     float scale, int in_dtype, int acc_dtype,
+                                     cpattn_stream_t stream);
+
+/*
  * cpattn_merge -- exact merge of two partial attention results over disjoint key sets
  * (the Ring Attention step: each rank folds each arriving K/V chunk's partial into its
  * running result with the online softmax, Fig. 3):
@@ -118,6 +158,18 @@ CPATTN_API int cpattn_merge(const void* o_a, const float* lse_a, const void* o_b
  */
 CPATTN_API int cpattn_seq2head(const void* src, void* dst, int P, int S_local, int H, int D,
                     int elem_bytes, cpattn_stream_t stream);
+
+/*
+ * cpattn_seq2head_qkv -- cpattn_seq2head of Q, K and V in one launch (the three
+ * sequence->head all-to-alls that precede Ulysses attention, Fig. 4; the serving blog's
+ * Cosmos 3 plan issues three all-to-alls per transformer layer).  Each of (q -> qh),
+ * (k -> kh), (v -> vh) is exactly cpattn_seq2head with the same P, S_local, H, D and
+ * elem_bytes; no destination may overlap any source or another destination.
+ * Errors: as cpattn_seq2head.
+ */
+CPATTN_API int cpattn_seq2head_qkv(const void* q, const void* k, const void* v, void* qh, void* kh,
+                                   void* vh, int P, int S_local, int H, int D, int elem_bytes,
+                                   cpattn_stream_t stream);
 
 /*
  * cpattn_head2seq -- the Ulysses second all-to-all (Fig. 4), exact inverse of

@@ -73,6 +73,34 @@ def test_fwd_argument_errors(L):
     assert fwd(L, B_=70000) == B.ERR_SHAPE
 
 
+def test_fwd_accumulate_argument_errors(L):
+    vp = ctypes.c_void_p
+
+    def acc(lse=FAKE, din=0, dout=0, D=128):
+        return L.cpattn_fwd_accumulate(vp(FAKE), vp(FAKE), vp(FAKE), vp(FAKE),
+                                       vp(lse) if lse else None, 1, 2, 8, 8, D, 0.1, din, dout,
+                                       None)
+
+    assert acc(lse=0) == B.ERR_NULL  # the running LSE is required
+    assert acc(din=1, dout=1) == B.ERR_UNSUPPORTED  # tensor-core path only
+    assert acc(D=96) == B.ERR_UNSUPPORTED
+    assert acc(dout=3) == B.ERR_UNSUPPORTED
+
+
+def test_ulysses_fwd_argument_errors(L):
+    vp = ctypes.c_void_p
+
+    def uf(P=2, S_l=32, H=4, D=128, dout=0, q=FAKE):
+        return L.cpattn_ulysses_fwd(vp(q) if q else None, vp(FAKE), vp(FAKE), vp(FAKE), None, P,
+                                    S_l, H, D, 0.1, dout, None)
+
+    assert uf(H=5) == B.ERR_SHAPE          # H % P
+    assert uf(S_l=24) == B.ERR_UNSUPPORTED  # 16-row boxes would straddle two shards
+    assert uf(D=96) == B.ERR_UNSUPPORTED
+    assert uf(q=0) == B.ERR_NULL
+    assert uf(q=FAKE + 8) == B.ERR_ALIGN
+
+
 def test_merge_argument_errors(L):
     vp = ctypes.c_void_p
     base = [vp(FAKE), vp(FAKE + 0x100000), vp(FAKE + 0x200000), vp(FAKE + 0x300000),
@@ -101,6 +129,18 @@ def test_permute_argument_errors(L):
         assert fn(None, d, 2, 4, 16, 128, 2, None) == B.ERR_NULL
         assert fn(vp(FAKE + 4), d, 2, 4, 16, 128, 2, None) == B.ERR_ALIGN
         assert fn(s, vp(FAKE + 64), 2, 4, 16, 128, 2, None) == B.ERR_SHAPE  # overlap
+
+
+def test_seq2head_qkv_argument_errors(L):
+    vp = ctypes.c_void_p
+    big = 0x1000000
+    ptrs = [vp(FAKE + i * big) for i in range(6)]
+    f = L.cpattn_seq2head_qkv
+    assert f(*ptrs, 3, 4, 16, 128, 2, None) == B.ERR_SHAPE  # H % P
+    assert f(None, *ptrs[1:], 2, 4, 16, 128, 2, None) == B.ERR_NULL
+    # kh overlapping vh
+    bad = ptrs[:4] + [vp(FAKE + 5 * big + 32)] + ptrs[5:]
+    assert f(*bad, 2, 4, 16, 128, 2, None) == B.ERR_SHAPE
 
 
 def test_selftest_limit_checked(L):

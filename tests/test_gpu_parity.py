@@ -69,6 +69,18 @@ def test_permutes_ulysses_full_size_bit_exact():
     assert torch.equal(bits(back).cpu(), src_bits)
 
 
+@pytest.mark.parametrize("P,S_l,H,D", [(2, 3, 4, 8), (8, 5520, 16, 128), (3, 7, 6, 16)])
+def test_seq2head_qkv_batched_bit_exact(P, S_l, H, D):
+    g = torch.Generator().manual_seed(P + S_l)
+    srcs = [torch.randint(-32768, 32768, (P, S_l, H, D), generator=g, dtype=torch.int32).to(torch.int16)
+            for _ in range(3)]
+    dev = [t.view(torch.bfloat16).to(DEV) for t in srcs]
+    outs = cp.seq2head_qkv(*dev, P)
+    torch.cuda.synchronize()
+    for src_bits, o in zip(srcs, outs):
+        np.testing.assert_array_equal(bits(o).cpu().numpy(), ref.seq2head(src_bits.numpy(), P))
+
+
 # ----------------------------------------------------------------------------- merge
 
 
@@ -175,6 +187,47 @@ def test_bf16_shapes_match_oracle(shape):
     assert rel_l2(o32, o_ref) < 1e-2
 
 
+@pytest.mark.parametrize("shape,split", [((1, 2, 130, 300, 128), 170), ((2, 1, 257, 129, 64), 1),
+                                         ((1, 3, 17, 513, 128), 384)])
+@pytest.mark.parametrize("acc", [torch.bfloat16, torch.float32])
+def test_fused_ring_accumulate_matches_oracle(shape, split, acc):
+    Bn, H, Sq, Skv, D = shape
+    q, k, v = W.random_case(Skv + split, Bn, H, Sq, Skv, D)
+    scale = 1.0 / math.sqrt(D)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    # start from an empty accumulator holding garbage (NaN) and LSE = -inf
+    o_acc = torch.full((Bn, Sq, H, D), float("nan"), dtype=acc, device=DEV)
+    l_acc = torch.full((Bn, H, Sq), -math.inf, device=DEV)
+    cp.fwd_accumulate(qd, kd[:, :split].contiguous(), vd[:, :split].contiguous(), o_acc, l_acc,
+                      scale=scale)
+    cp.fwd_accumulate(qd, kd[:, split:].contiguous(), vd[:, split:].contiguous(), o_acc, l_acc,
+                      scale=scale)
+    torch.cuda.synchronize()
+    o_ref, l_ref = ref.attention(q, k, v, scale)
+    check_o(o_acc, o_ref, "bf16_out" if acc == torch.bfloat16 else "bf16_in", f"{shape} fused ring")
+    check_lse(l_acc, l_ref, f"{shape} fused ring")
+    # the fused step equals partial + separate merge
+    oa, la = cp.fwd(qd, kd[:, :split].contiguous(), vd[:, :split].contiguous(), scale=scale,
+                    out_dtype=torch.float32)
+    ob, lb = cp.fwd(qd, kd[:, split:].contiguous(), vd[:, split:].contiguous(), scale=scale,
+                    out_dtype=torch.float32)
+    om, lm = cp.merge(oa, la, ob, lb)
+    torch.cuda.synchronize()
+    assert (l_acc - lm).abs().max().item() < 1e-5
+    if acc == torch.float32:
+        assert (o_acc - om).abs().max().item() < 1e-5
+
+
+def test_accumulate_empty_chunk_is_identity():
+    q, k, v = (t.to(DEV) for t in W.random_case(3, 1, 2, 40, 50, 128))
+    o, l = cp.fwd(q, k, v, out_dtype=torch.float32)
+    o0, l0 = o.clone(), l.clone()
+    e = torch.empty(1, 0, 2, 128, dtype=torch.bfloat16, device=DEV)
+    cp.fwd_accumulate(q, e, e, o, l)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o0) and torch.equal(l, l0)
+
+
 def test_bf16_large_logits_stable():
     q, k, v = W.random_case(5, 1, 2, 300, 700, 128, sigma_qk=3.0)
     scale = 1.0 / math.sqrt(128)
@@ -234,6 +287,43 @@ def test_invariants_on_gpu():
     assert ((l3 - l1) - math.log(2)).abs().max().item() < 1e-4
 
 
+# ----------------------------------------------------------------------------- fused Ulysses
+
+
+@pytest.mark.parametrize("P,S_l,H,D", [(2, 32, 4, 128), (3, 48, 6, 128), (1, 144, 2, 64),
+                                       (4, 400, 8, 64), (8, 16, 16, 128)])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_fused_ulysses_equals_permute_path(P, S_l, H, D, out_dtype):
+    g = torch.Generator().manual_seed(P * 100 + S_l)
+    shards = [W.randn((P, S_l, H, D), g, 1.0, "bf16").to(DEV) for _ in range(3)]
+    out_f, lse_f = cp.ulysses_fwd(*shards, P, out_dtype=out_dtype)
+    qh, kh, vh = (cp.seq2head(t, P) for t in shards)
+    oh, lse_u = cp.fwd(qh, kh, vh, out_dtype=out_dtype)
+    out_u = cp.head2seq(oh, P)
+    torch.cuda.synchronize()
+    # same tiles, same arithmetic: identical bits
+    assert torch.equal(out_f, out_u) and torch.equal(lse_f, lse_u)
+    # and the single-device meaning: attention over the concatenated shards
+    full = lambda t: t.cpu().reshape(1, P * S_l, H, D)
+    o_ref, l_ref = ref.attention(full(shards[0]), full(shards[1]), full(shards[2]), 1 / math.sqrt(D))
+    check_o(out_f.reshape(1, P * S_l, H, D), o_ref,
+            "bf16_out" if out_dtype == torch.bfloat16 else "bf16_in", "fused ulysses")
+    hp = H // P
+    check_lse(lse_f.cpu().reshape(H, P * S_l), l_ref[0].reshape(H, P * S_l), "fused ulysses")
+
+
+def test_fused_ulysses_full_size_bit_identical():
+    w = W.WORKLOADS[4]
+    x = W.make_inputs(w)
+    P = w.P
+    q, k, v = (x[n].to(DEV) for n in ("q", "k", "v"))
+    out_f, lse_f = cp.ulysses_fwd(q, k, v, P)
+    plan = UlyssesPlan(P, w.Sq // P, w.H * P, w.D)
+    out_u, lse_u = plan.run(q, k, v)
+    torch.cuda.synchronize()
+    assert torch.equal(out_f, out_u) and torch.equal(lse_f, lse_u)
+
+
 # ----------------------------------------------------------------------------- the five workloads
 
 
@@ -267,15 +357,19 @@ def test_workload3_ring_step():
     vc = [v[:, a:b].contiguous() for a, b in zip(bounds, bounds[1:])]
     o_ring, l_ring = cp.ring_attention(q, kc, vc, scale=w.softmax_scale)
     o_ring32, l_ring32 = cp.ring_attention(q, kc, vc, scale=w.softmax_scale, acc_dtype=torch.float32)
+    o_unf32, l_unf32 = cp.ring_attention(q, kc, vc, scale=w.softmax_scale,
+                                         acc_dtype=torch.float32, fused=False)
     o_one, l_one = cp.fwd(q, k, v, scale=w.softmax_scale, out_dtype=torch.float32)
     torch.cuda.synchronize()
     rows = W.sample_rows(w.B, w.H, w.Sq, 2048, seed=3)
     _sampled(x["q"], x["k"], x["v"], w.softmax_scale, o_ring.cpu(), l_ring.cpu(), rows, "bf16_out", "ring bf16")
     _sampled(x["q"], x["k"], x["v"], w.softmax_scale, o_ring32.cpu(), l_ring32.cpu(), rows, "bf16_in", "ring fp32")
     _sampled(x["q"], x["k"], x["v"], w.softmax_scale, o_one.cpu(), l_one.cpu(), rows, "bf16_in", "single pass")
-    # whole-tensor property: ring result == single-pass result
+    # whole-tensor properties: ring result == single-pass result; fused == separate merge
     assert (o_ring32 - o_one).abs().max().item() < 1e-3
     assert (l_ring32 - l_one).abs().max().item() < 1e-4
+    assert (o_ring32 - o_unf32).abs().max().item() < 1e-5
+    assert (l_ring32 - l_unf32).abs().max().item() < 1e-5
 
 
 def test_workload4_ulysses():
@@ -285,7 +379,10 @@ def test_workload4_ulysses():
     q, k, v = (x[n].to(DEV) for n in ("q", "k", "v"))
     plan = UlyssesPlan(P, w.Sq // P, w.H * P, w.D)
     out, lse = plan.run(q, k, v, scale=w.softmax_scale)
+    plan_b = UlyssesPlan(P, w.Sq // P, w.H * P, w.D, batched=True)
+    out_b, lse_b = plan_b.run(q, k, v, scale=w.softmax_scale)
     torch.cuda.synchronize()
+    assert torch.equal(bits(out_b), bits(out)) and torch.equal(lse_b, lse)  # same kernels, same bits
     # the permutes are bit-exact against the oracle's re-partition
     for name, dev_buf in (("q", plan.qh), ("k", plan.kh), ("v", plan.vh)):
         np.testing.assert_array_equal(bits(dev_buf).cpu().numpy(),
