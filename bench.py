@@ -231,6 +231,7 @@ def run_ours(args, world, rank, local):
     else:
         # ---- auxiliary HBM-bound kernels, timed alone (L2 flushed before each launch)
         aux = aux_kernels(cp, w, q, plan, dev, stream)
+        aux["next"] = next_paths(cp, w, q, k, v, plan, dev, stream)
         # ---- end to end through the public API with host buffers
         e2e = e2e_run(cp, UlyssesPlan, w, x, dev, stream, args)
 
@@ -337,6 +338,53 @@ def aux_kernels(cp, w, q, plan, dev, stream):
     out["l2"] = ("512 MB buffer written then read before each burst; each burst's buffers "
                  "exceed L2")
     return out
+
+
+def next_paths(cp, w, q, k, v, plan, dev, stream):
+    """The fused forms of the path, timed alone after an L2 flush (median of 5):
+    Ulysses in one kernel, the batched Q/K/V seq2head, and one rank's Ring Attention step
+    (Q slice of 5520 tokens over 8 K/V chunks of 5520, 16 heads) with the merge fused into
+    the attention epilogue versus separate partials + merge kernel."""
+    peaks = measured_peaks()
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    def timed(fn, reps=5):
+        ts = []
+        for _ in range(reps):
+            flush_l2(flush)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    res = {}
+    ms = timed(lambda: cp.ulysses_fwd(q, k, v, w.P, out=plan.out, lse=plan.lse))
+    res["ulysses_fused"] = {"ms": round(ms, 4), "TFLOP/s": round(w.attn_flops / ms / 1e9, 2),
+                            "what": "seq2head x3 + attention + head2seq as one kernel"}
+    ms = timed(lambda: cp.seq2head_qkv(q, k, v, w.P, out=(plan.qh, plan.kh, plan.vh)))
+    nbytes = 3 * 2 * q.numel() * q.element_size()
+    res["seq2head_qkv"] = {"ms": round(ms, 4), "bytes": nbytes,
+                           "GB/s": round(nbytes / ms / 1e6, 1),
+                           "frac_of_hbm": round(nbytes / ms / 1e6 / peaks["hbm_gbs"], 4)}
+    w3 = W.WORKLOADS[3]
+    x3 = W.make_inputs(w3)
+    q3, k3, v3 = (x3[n].to(dev) for n in ("q", "k", "v"))
+    bounds = [0]
+    for c in x3["chunks"]:
+        bounds.append(bounds[-1] + c)
+    kc = [k3[:, a:b].contiguous() for a, b in zip(bounds, bounds[1:])]
+    vc = [v3[:, a:b].contiguous() for a, b in zip(bounds, bounds[1:])]
+    ms_f = timed(lambda: cp.ring_attention(q3, kc, vc, scale=w3.softmax_scale, fused=True))
+    ms_u = timed(lambda: cp.ring_attention(q3, kc, vc, scale=w3.softmax_scale, fused=False))
+    res["ring_step"] = {
+        "workload": "Q [1][5520][16][128] over 8 K/V chunks of 5520 tokens, bf16 accumulator",
+        "fused_ms": round(ms_f, 4), "fused_TFLOP/s": round(w3.attn_flops / ms_f / 1e9, 2),
+        "unfused_ms": round(ms_u, 4), "unfused_TFLOP/s": round(w3.attn_flops / ms_u / 1e9, 2),
+        "launches_fused": 8, "launches_unfused": 15}
+    return res
 
 
 def e2e_run(cp, UlyssesPlan, w, x, dev, stream, args):

@@ -174,14 +174,16 @@ int cpattn_ulysses_fwd(const void* q, const void* k, const void* v, void* out, f
     return CPATTN_ERR_ALIGN;
   int* err = device_error_word();
   if (err == nullptr) return CPATTN_ERR_CUDA;
-  CUtensorMap tq, tk, tv;
-  if (!encode_bshd_bf16(&tq, q, P, S_local, H, D, 16) ||
-      !encode_bshd_bf16(&tk, k, P, S_local, H, D, 16) ||
-      !encode_bshd_bf16(&tv, v, P, S_local, H, D, 16))
+  CUtensorMap tq, tk, tv, tq16, tk16, tv16;
+  if (!encode_bshd_bf16(&tq, q, P, S_local, H, D) || !encode_bshd_bf16(&tk, k, P, S_local, H, D) ||
+      !encode_bshd_bf16(&tv, v, P, S_local, H, D) ||
+      !encode_bshd_bf16(&tq16, q, P, S_local, H, D, 16) ||
+      !encode_bshd_bf16(&tk16, k, P, S_local, H, D, 16) ||
+      !encode_bshd_bf16(&tv16, v, P, S_local, H, D, 16))
     return CPATTN_ERR_CUDA;
   const float scale_log2 = float(double(scale) * 1.4426950408889634074);
   return cuda_status(cpattn::launch_ulysses_fwd_sm100(
-      tq, tk, tv, out, lse, P, S_local, H, D, scale_log2, cpattn::kRescaleLog2,
+      tq, tk, tv, tq16, tk16, tv16, out, lse, P, S_local, H, D, scale_log2, cpattn::kRescaleLog2,
       out_dtype == CPATTN_F32, err, cpattn::kDefaultWaitLimit,
       reinterpret_cast<cudaStream_t>(stream)));
 }

@@ -86,7 +86,10 @@ template <int D, bool kOutF32, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
-                          const __grid_constant__ CUtensorMap tm_v, void* __restrict__ out,
+                          const __grid_constant__ CUtensorMap tm_v,
+                          const __grid_constant__ CUtensorMap tm_q16,
+                          const __grid_constant__ CUtensorMap tm_k16,
+                          const __grid_constant__ CUtensorMap tm_v16, void* __restrict__ out,
                           float* __restrict__ lse, int H, int Sq, int Skv, float scale_log2,
                           float rescale_log2, int s_local, int* err, long long wait_limit) {
   using G = Geometry<D>;
@@ -96,7 +99,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // sequence is read straight from the sequence shards [P][S_l][H*P][D] (token t lives in
   // shard t / S_l, row t % S_l) with 16-row TMA boxes, so no box crosses a shard boundary
   // (S_l % 16 == 0), and O goes back to the same sharded layout: the all-to-alls become
-  // addressing.
+  // addressing.  A tile inside one shard is a single 128-row box (tm_q/k/v); only tiles
+  // that straddle a shard boundary use the 16-row maps (tm_q16/k16/v16).
   constexpr bool kShard = kMode == kSharded;
   extern __shared__ uint8_t smem_raw[];
   __shared__ Barriers bars;
@@ -134,6 +138,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
+    if (kShard) {
+      tma_prefetch_desc(&tm_q16);
+      tma_prefetch_desc(&tm_k16);
+      tma_prefetch_desc(&tm_v16);
+    }
   }
   if (warp == kWarpMma) {
     tmem_alloc(smem_u32(&tmem_base_sh), kTmemCols);
@@ -349,18 +358,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (elect_one()) {
       // one 128-row tile starting at token t0 into `dst`: a 64-column box per 128-byte
       // column block; sharded inputs take eight 16-row boxes, each inside one rank shard
-      auto load_tile = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, int t0) {
+      auto load_tile = [&](const CUtensorMap* map, const CUtensorMap* map16, uint32_t dst,
+                           uint32_t bar, int t0) {
+        if constexpr (!kShard) {
 #pragma unroll
-        for (int bx = 0; bx < G::kBoxes; ++bx) {
-          if constexpr (!kShard) {
+          for (int bx = 0; bx < G::kBoxes; ++bx)
             tma_load_4d(dst + bx * G::kBoxBytes, map, bar, bx * G::kBox, head_coord, t0, b);
+        } else {
+          int r = t0 / s_local;  // rank shard (== P past the end: zero-filled)
+          int sr = t0 - r * s_local;
+          if (sr + kBlockN <= s_local) {
+#pragma unroll
+            for (int bx = 0; bx < G::kBoxes; ++bx)
+              tma_load_4d(dst + bx * G::kBoxBytes, map, bar, bx * G::kBox, head_coord, sr, r);
           } else {
 #pragma unroll 1
             for (int i = 0; i < kBlockN / 16; ++i) {
-              const int t = t0 + 16 * i;
-              const int r = t / s_local;  // rank shard (== P past the end: zero-filled)
-              tma_load_4d(dst + bx * G::kBoxBytes + i * 16 * 128, map, bar, bx * G::kBox,
-                          head_coord, t - r * s_local, r);
+#pragma unroll
+              for (int bx = 0; bx < G::kBoxes; ++bx)
+                tma_load_4d(dst + bx * G::kBoxBytes + i * 16 * 128, map16, bar, bx * G::kBox,
+                            head_coord, sr, r);
+              sr += 16;
+              if (sr >= s_local) {
+                sr -= s_local;
+                ++r;
+              }
             }
           }
         }
@@ -369,7 +391,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(bar_q, 2 * G::kTileBytes);
 #pragma unroll
       for (int t = 0; t < 2; ++t)
-        load_tile(&tm_q, smem_base + G::kOffQ + t * G::kTileBytes, bar_q, q_first + t * kBlockM);
+        load_tile(&tm_q, &tm_q16, smem_base + G::kOffQ + t * G::kTileBytes, bar_q,
+                  q_first + t * kBlockM);
       int issued = 0;
       for (int use = 0; use < 2 * n_kv; ++use) {
         const int slot = use % kSlots;
@@ -377,9 +400,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(smem_u32(&bars.empty[slot]), ph ^ 1u, abort_flag, err, wait_limit)) break;
         const uint32_t bar_f = smem_u32(&bars.full[slot]);
         mbar_arrive_expect_tx(bar_f, G::kTileBytes);
-        const CUtensorMap* map = (use & 1) ? &tm_v : &tm_k;
-        load_tile(map, smem_base + G::kOffSlots + slot * G::kTileBytes, bar_f,
-                  (use >> 1) * kBlockN);
+        load_tile((use & 1) ? &tm_v : &tm_k, (use & 1) ? &tm_v16 : &tm_k16,
+                  smem_base + G::kOffSlots + slot * G::kTileBytes, bar_f, (use >> 1) * kBlockN);
         issued = use + 1;
       }
       // drain: every issued copy must have landed before the CTA's shared memory is
@@ -472,8 +494,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D, bool kOutF32, int kMode>
-cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* out,
-                   float* lse, dim3 grid, int H, int Sq, int Skv, float scale_log2,
+cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                   const CUtensorMap& tq16, const CUtensorMap& tk16, const CUtensorMap& tv16,
+                   void* out, float* lse, dim3 grid, int H, int Sq, int Skv, float scale_log2,
                    float rescale_log2, int s_local, int* err, long long wait_limit,
                    cudaStream_t stream) {
   using G = Geometry<D>;
@@ -481,48 +504,54 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        G::kDynSmem);
   if (e != cudaSuccess) return e;
-  kernel<<<grid, kThreads, G::kDynSmem, stream>>>(tq, tk, tv, out, lse, H, Sq, Skv, scale_log2,
-                                                   rescale_log2, s_local, err, wait_limit);
+  kernel<<<grid, kThreads, G::kDynSmem, stream>>>(tq, tk, tv, tq16, tk16, tv16, out, lse, H, Sq,
+                                                   Skv, scale_log2, rescale_log2, s_local, err,
+                                                   wait_limit);
   return cudaGetLastError();
 }
 
 template <int D, int kMode>
-cudaError_t launch_o(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* out,
+cudaError_t launch_o(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                     const CUtensorMap& tq16, const CUtensorMap& tk16, const CUtensorMap& tv16,
+                     void* out,
                      float* lse, dim3 grid, int H, int Sq, int Skv, float scale_log2,
                      float rescale_log2, int s_local, bool out_f32, int* err, long long wait_limit,
                      cudaStream_t stream) {
-  return out_f32 ? launch<D, true, kMode>(tq, tk, tv, out, lse, grid, H, Sq, Skv, scale_log2,
+  return out_f32 ? launch<D, true, kMode>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv, scale_log2,
                                           rescale_log2, s_local, err, wait_limit, stream)
-                 : launch<D, false, kMode>(tq, tk, tv, out, lse, grid, H, Sq, Skv, scale_log2,
+                 : launch<D, false, kMode>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv, scale_log2,
                                            rescale_log2, s_local, err, wait_limit, stream);
 }
 
 template <int D>
-cudaError_t launch_m(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* out,
+cudaError_t launch_m(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                     const CUtensorMap& tq16, const CUtensorMap& tk16, const CUtensorMap& tv16,
+                     void* out,
                      float* lse, dim3 grid, int H, int Sq, int Skv, float scale_log2,
                      float rescale_log2, int s_local, bool out_f32, int mode, int* err,
                      long long wait_limit, cudaStream_t stream) {
   switch (mode) {
     case kAccum:
-      return launch_o<D, kAccum>(tq, tk, tv, out, lse, grid, H, Sq, Skv, scale_log2, rescale_log2,
+      return launch_o<D, kAccum>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv, scale_log2, rescale_log2,
                                  s_local, out_f32, err, wait_limit, stream);
     case kSharded:
-      return launch_o<D, kSharded>(tq, tk, tv, out, lse, grid, H, Sq, Skv, scale_log2,
+      return launch_o<D, kSharded>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv, scale_log2,
                                    rescale_log2, s_local, out_f32, err, wait_limit, stream);
     default:
-      return launch_o<D, kPlain>(tq, tk, tv, out, lse, grid, H, Sq, Skv, scale_log2, rescale_log2,
+      return launch_o<D, kPlain>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv, scale_log2, rescale_log2,
                                  s_local, out_f32, err, wait_limit, stream);
   }
 }
 
 cudaError_t launch_any(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tq16, const CUtensorMap& tk16, const CUtensorMap& tv16,
                        void* out, float* lse, dim3 grid, int H, int Sq, int Skv, int D,
                        float scale_log2, float rescale_log2, int s_local, bool out_f32, int mode,
                        int* err, long long wait_limit, cudaStream_t stream) {
   if (D == 128)
-    return launch_m<128>(tq, tk, tv, out, lse, grid, H, Sq, Skv, scale_log2, rescale_log2, s_local,
+    return launch_m<128>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv, scale_log2, rescale_log2, s_local,
                          out_f32, mode, err, wait_limit, stream);
-  return launch_m<64>(tq, tk, tv, out, lse, grid, H, Sq, Skv, scale_log2, rescale_log2, s_local,
+  return launch_m<64>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv, scale_log2, rescale_log2, s_local,
                       out_f32, mode, err, wait_limit, stream);
 }
 
@@ -534,18 +563,21 @@ cudaError_t launch_attn_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
                                   bool out_f32, bool accumulate, int* err, long long wait_limit,
                                   cudaStream_t stream) {
   const dim3 grid((Sq + 2 * kBlockM - 1) / (2 * kBlockM), H, B);
-  return launch_any(tq, tk, tv, out, lse, grid, H, Sq, Skv, D, scale_log2, rescale_log2, 0,
+  return launch_any(tq, tk, tv, tq, tk, tv, out, lse, grid, H, Sq, Skv, D, scale_log2, rescale_log2, 0,
                     out_f32, accumulate ? kAccum : kPlain, err, wait_limit, stream);
 }
 
 cudaError_t launch_ulysses_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
-                                     const CUtensorMap& tv, void* out, float* lse, int P,
+                                     const CUtensorMap& tv, const CUtensorMap& tq16,
+                                     const CUtensorMap& tk16, const CUtensorMap& tv16, void* out,
+                                     float* lse, int P,
                                      int S_local, int H, int D, float scale_log2,
                                      float rescale_log2, bool out_f32, int* err,
                                      long long wait_limit, cudaStream_t stream) {
   const int S = P * S_local, Hp = H / P;
   const dim3 grid((S + 2 * kBlockM - 1) / (2 * kBlockM), Hp, P);
-  return launch_any(tq, tk, tv, out, lse, grid, Hp, S, S, D, scale_log2, rescale_log2, S_local,
+  return launch_any(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, Hp, S, S, D, scale_log2,
+                    rescale_log2, S_local,
                     out_f32, kSharded, err, wait_limit, stream);
 }
 

@@ -19,10 +19,13 @@ cudaError_t launch_attn_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
                                   bool out_f32, bool accumulate, int* err, long long wait_limit,
                                   cudaStream_t stream);
 
-// Ulysses fused: q/k/v/out are [P][S_local][H][D] rank shards (tensor maps with a
-// 64 x 1 x 16 x 1 box over dims (D, H, S_local, P)); LSE is [P][H/P][P*S_local].
+// Ulysses fused: q/k/v/out are [P][S_local][H][D] rank shards, each described by two tensor
+// maps over dims (D, H, S_local, P): a 64 x 1 x 128 x 1 box and a 64 x 1 x 16 x 1 box (for
+// tiles that straddle two shards); LSE is [P][H/P][P*S_local].
 cudaError_t launch_ulysses_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
-                                     const CUtensorMap& tv, void* out, float* lse, int P,
+                                     const CUtensorMap& tv, const CUtensorMap& tq16,
+                                     const CUtensorMap& tk16, const CUtensorMap& tv16, void* out,
+                                     float* lse, int P,
                                      int S_local, int H, int D, float scale_log2,
                                      float rescale_log2, bool out_f32, int* err,
                                      long long wait_limit, cudaStream_t stream);
