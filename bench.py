@@ -377,13 +377,34 @@ def next_paths(cp, w, q, k, v, plan, dev, stream):
         bounds.append(bounds[-1] + c)
     kc = [k3[:, a:b].contiguous() for a, b in zip(bounds, bounds[1:])]
     vc = [v3[:, a:b].contiguous() for a, b in zip(bounds, bounds[1:])]
+    n_split = cp.split_suggest(1, w3.H, w3.Sq, x3["chunks"][0])
     ms_f = timed(lambda: cp.ring_attention(q3, kc, vc, scale=w3.softmax_scale, fused=True))
     ms_u = timed(lambda: cp.ring_attention(q3, kc, vc, scale=w3.softmax_scale, fused=False))
+    ms_s = timed(lambda: cp.ring_attention(q3, kc, vc, scale=w3.softmax_scale, fused=True,
+                                           n_split=n_split))
+    # AllGather-KV-like: a short query slice (512 tokens, 16 heads) against all 44160 keys --
+    # 32 CTAs for 148 SMs, the case split-KV is for
+    g = torch.Generator(device="cpu").manual_seed(41)
+    qs = W.randn((1, 512, 16, 128), g, 1.0, "bf16").to(dev)
+    ks = k3.reshape(1, -1, 16, 128)[:, :44160].contiguous()
+    vs = v3.reshape(1, -1, 16, 128)[:, :44160].contiguous()
+    flops_s = 4.0 * 16 * 512 * 44160 * 128
+    ns = cp.split_suggest(1, 16, 512, 44160)
+    ms_1 = timed(lambda: cp.fwd(qs, ks, vs))
+    ws = torch.empty(cp.split_workspace_bytes(1, 16, 512, 128, ns), dtype=torch.uint8, device=dev)
+    ms_n = timed(lambda: cp.fwd_split(qs, ks, vs, n_split=ns, workspace=ws))
+    res["split_kv_short_q"] = {"workload": "Q [1][512][16][128] over 44160 keys", "n_split": ns,
+                               "single_ms": round(ms_1, 4),
+                               "single_TFLOP/s": round(flops_s / ms_1 / 1e9, 2),
+                               "split_ms": round(ms_n, 4),
+                               "split_TFLOP/s": round(flops_s / ms_n / 1e9, 2)}
     res["ring_step"] = {
         "workload": "Q [1][5520][16][128] over 8 K/V chunks of 5520 tokens, bf16 accumulator",
         "fused_ms": round(ms_f, 4), "fused_TFLOP/s": round(w3.attn_flops / ms_f / 1e9, 2),
         "unfused_ms": round(ms_u, 4), "unfused_TFLOP/s": round(w3.attn_flops / ms_u / 1e9, 2),
-        "launches_fused": 8, "launches_unfused": 15}
+        "split_kv": n_split, "split_ms": round(ms_s, 4),
+        "split_TFLOP/s": round(w3.attn_flops / ms_s / 1e9, 2),
+        "launches_fused": 8, "launches_unfused": 15, "launches_split": 16}
     return res
 
 

@@ -17,6 +17,9 @@ from ._binding import (  # noqa: F401
     device_error,
     fwd,
     fwd_accumulate,
+    fwd_split,
+    split_suggest,
+    split_workspace_bytes,
     ulysses_fwd,
     head2seq,
     lib,

@@ -49,6 +49,11 @@ def lib() -> ctypes.CDLL:
             L.cpattn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
             L.cpattn_fwd_accumulate.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
             L.cpattn_ulysses_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+            L.cpattn_fwd_split.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp,
+                                           ctypes.c_size_t, vp]
+            L.cpattn_fwd_split_workspace.argtypes = [i, i, i, i, i, i]
+            L.cpattn_fwd_split_workspace.restype = ctypes.c_size_t
+            L.cpattn_split_suggest.argtypes = [i, i, i, i]
             L.cpattn_merge.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
             L.cpattn_seq2head.argtypes = [vp, vp, i, i, i, i, i, vp]
             L.cpattn_head2seq.argtypes = [vp, vp, i, i, i, i, i, vp]
@@ -59,7 +64,8 @@ def lib() -> ctypes.CDLL:
             L.cpattn_selftest_wait_timeout.argtypes = [ll, vp]
             L.cpattn_version.argtypes = []
             L.cpattn_selftest_exp2.argtypes = [vp, vp, i, vp]
-            for name in ("cpattn_fwd", "cpattn_fwd_accumulate", "cpattn_ulysses_fwd", "cpattn_merge", "cpattn_seq2head_qkv", "cpattn_seq2head", "cpattn_head2seq",
+            for name in ("cpattn_fwd", "cpattn_fwd_accumulate", "cpattn_ulysses_fwd",
+                         "cpattn_fwd_split", "cpattn_split_suggest", "cpattn_merge", "cpattn_seq2head_qkv", "cpattn_seq2head", "cpattn_head2seq",
                          "cpattn_device_error", "cpattn_selftest_wait_timeout", "cpattn_version",
                          "cpattn_selftest_exp2"):
                 getattr(L, name).restype = ctypes.c_int
@@ -146,6 +152,42 @@ def ulysses_fwd(q, k, v, P, out=None, lse=None, scale=None, out_dtype=None, want
     st = lib().cpattn_ulysses_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), P, S_l, H, D,
                                   float(scale), _dtype_code(out.dtype), _stream(stream))
     _check(st, "cpattn_ulysses_fwd")
+    return out, lse
+
+
+def split_workspace_bytes(B, H, Sq, D, n_split, out_dtype=torch.bfloat16) -> int:
+    return int(lib().cpattn_fwd_split_workspace(B, H, Sq, D, n_split, _dtype_code(out_dtype)))
+
+
+def split_suggest(B, H, Sq, Skv) -> int:
+    return int(lib().cpattn_split_suggest(B, H, Sq, Skv))
+
+
+def fwd_split(q, k, v, out=None, lse=None, scale=None, out_dtype=None, accumulate=False,
+              n_split=None, workspace=None, stream=None):
+    """Split-KV attention: ``n_split`` key ranges computed as separate CTAs, their partials
+    folded exactly (into the running (out, lse) when ``accumulate``).  ``workspace`` is a
+    uint8 CUDA tensor of at least ``split_workspace_bytes(...)`` bytes (allocated here when
+    omitted -- by PyTorch; the library allocates nothing)."""
+    B_, Sq, H, D = q.shape
+    Skv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty((B_, Sq, H, D), dtype=out_dtype or q.dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B_, H, Sq), dtype=torch.float32, device=q.device)
+    if n_split is None:
+        n_split = split_suggest(B_, H, Sq, Skv)
+    need = split_workspace_bytes(B_, H, Sq, D, n_split, out.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    _need_cuda(q, k, v, out, lse, workspace)
+    st = lib().cpattn_fwd_split(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B_, H, Sq, Skv,
+                                D, float(scale), _dtype_code(out.dtype), 1 if accumulate else 0,
+                                int(n_split), _ptr(workspace), workspace.numel(),
+                                _stream(stream))
+    _check(st, "cpattn_fwd_split")
     return out, lse
 
 

@@ -133,7 +133,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* out, float* lse,
     const float scale_log2 = float(double(scale) * 1.4426950408889634074);
     return cuda_status(cpattn::launch_attn_fwd_sm100(
         tq, tk, tv, out, lse, B, H, Sq, Skv, D, scale_log2, cpattn::kRescaleLog2,
-        out_dtype == CPATTN_F32, accumulate, err, cpattn::kDefaultWaitLimit, st));
+        out_dtype == CPATTN_F32, accumulate, 1, err, cpattn::kDefaultWaitLimit, st));
   }
   // fp32 inputs: CUDA-core kernel
   return cuda_status(cpattn::launch_attn_fwd_f32(
@@ -156,6 +156,97 @@ int cpattn_fwd_accumulate(const void* q, const void* k, const void* v, void* o_a
                           int in_dtype, int acc_dtype, cpattn_stream_t stream) {
   return fwd_impl(q, k, v, o_acc, lse_acc, B, H, Sq, Skv, D, scale, in_dtype, acc_dtype, true,
                   stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+constexpr int kMaxSplit = 8;
+
+size_t split_o_bytes(int B, int H, int Sq, int D, int n, int es) {
+  const size_t o = size_t(n) * B * Sq * H * D * es;
+  return (o + 255) & ~size_t(255);
+}
+
+size_t split_ws_bytes(int B, int H, int Sq, int D, int n, int es) {
+  return split_o_bytes(B, H, Sq, D, n, es) + size_t(n) * B * H * Sq * sizeof(float);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t cpattn_fwd_split_workspace(int B, int H, int Sq, int D, int n_split, int out_dtype) {
+  const int es = elem_size(out_dtype);
+  if (B < 1 || H < 1 || Sq < 1 || D < 1 || n_split < 1 || n_split > kMaxSplit || es == 0)
+    return 0;
+  return n_split == 1 ? 0 : split_ws_bytes(B, H, Sq, D, n_split, es);
+}
+
+int cpattn_split_suggest(int B, int H, int Sq, int Skv) {
+  if (B < 1 || H < 1 || Sq < 1 || Skv < 1) return 1;
+  const long long ctas = (long long)((Sq + 255) / 256) * H * B;
+  const int sms = cpattn::sm_count();
+  const int n_kv = (Skv + 127) / 128;
+  if (ctas >= 4LL * sms) return 1;  // already four or more waves: little tail to recover
+  // modelled time per split count: waves of CTAs that each do 1/s of the key blocks, plus
+  // a per-CTA start-up (prologue, pipeline fill, epilogue) worth ~10 key blocks -- measured:
+  // a 352-CTA grid of 43-block CTAs gains nothing from two ranges -- and a combine pass of
+  // ~1 block per split
+  double best = 1e30;
+  int best_s = 1;
+  for (int sp = 1; sp <= kMaxSplit && n_kv / sp >= 4; ++sp) {
+    const long long waves = (ctas * sp + sms - 1) / sms;
+    const double t = double(waves) * (double(n_kv) / sp + 10.0) + (sp > 1 ? sp : 0);
+    if (t < best * 0.97) {
+      best = t;
+      best_s = sp;
+    }
+  }
+  return best_s;
+}
+
+int cpattn_fwd_split(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                     int H, int Sq, int Skv, int D, float scale, int out_dtype, int accumulate,
+                     int n_split, void* workspace, size_t workspace_bytes,
+                     cpattn_stream_t stream) {
+  if (n_split < 1 || n_split > kMaxSplit) return CPATTN_ERR_SHAPE;
+  const int n_kv = Skv > 0 ? (Skv + 127) / 128 : 0;
+  if (n_split > n_kv) n_split = n_kv > 0 ? n_kv : 1;  // every range holds a key block
+  if (n_split == 1)
+    return fwd_impl(q, k, v, out, lse, B, H, Sq, Skv, D, scale, CPATTN_BF16, out_dtype,
+                    accumulate != 0, stream);
+  // validate the call exactly as the single-pass form would (no launch yet)
+  if (B < 1 || H < 1 || Sq < 1 || D < 1) return CPATTN_ERR_SHAPE;
+  if (!(std::isfinite(scale) && scale > 0.f)) return CPATTN_ERR_SHAPE;
+  const int es = elem_size(out_dtype);
+  if (es == 0) return CPATTN_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return CPATTN_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535) return CPATTN_ERR_SHAPE;
+  if (!q || !k || !v || !out || !workspace) return CPATTN_ERR_NULL;
+  if (accumulate && lse == nullptr) return CPATTN_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      !aligned(workspace, 256) || (lse != nullptr && !aligned(lse, 4)))
+    return CPATTN_ERR_ALIGN;
+  if (workspace_bytes < split_ws_bytes(B, H, Sq, D, n_split, es)) return CPATTN_ERR_SHAPE;
+  int* err = device_error_word();
+  if (err == nullptr) return CPATTN_ERR_CUDA;
+  CUtensorMap tq, tk, tv;
+  if (!encode_bshd_bf16(&tq, q, B, Sq, H, D) || !encode_bshd_bf16(&tk, k, B, Skv, H, D) ||
+      !encode_bshd_bf16(&tv, v, B, Skv, H, D))
+    return CPATTN_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  void* part_o = workspace;
+  float* part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                             split_o_bytes(B, H, Sq, D, n_split, es));
+  const float scale_log2 = float(double(scale) * 1.4426950408889634074);
+  cudaError_t e = cpattn::launch_attn_fwd_sm100(
+      tq, tk, tv, part_o, part_lse, B, H, Sq, Skv, D, scale_log2, cpattn::kRescaleLog2,
+      out_dtype == CPATTN_F32, false, n_split, err, cpattn::kDefaultWaitLimit, st);
+  if (e != cudaSuccess) return CPATTN_ERR_CUDA;
+  return cuda_status(cpattn::launch_combine(part_o, part_lse, n_split, out, lse, B, H, Sq, D, es,
+                                            accumulate != 0, st));
 }
 
 int cpattn_ulysses_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int P,

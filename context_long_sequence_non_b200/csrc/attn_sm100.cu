@@ -91,7 +91,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                           const __grid_constant__ CUtensorMap tm_k16,
                           const __grid_constant__ CUtensorMap tm_v16, void* __restrict__ out,
                           float* __restrict__ lse, int H, int Sq, int Skv, float scale_log2,
-                          float rescale_log2, int s_local, int* err, long long wait_limit) {
+                          float rescale_log2, int s_local, int n_split, int* err,
+                          long long wait_limit) {
   using G = Geometry<D>;
   constexpr bool kAcc = kMode == kAccum;
   // kSharded: the DeepSpeed Ulysses path in one kernel.  The grid's z is the head group g
@@ -112,11 +113,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t smem_base = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int q_first = blockIdx.x * (2 * kBlockM);
+  // split-KV: blockIdx.x = (query tile pair) * n_split + split; split s takes a contiguous
+  // range of key blocks and writes its partial (O, LSE) to its own slice of out / lse
+  const int split = n_split > 1 ? int(blockIdx.x % unsigned(n_split)) : 0;
+  const int q_first = int(blockIdx.x / unsigned(n_split)) * (2 * kBlockM);
   const int h = blockIdx.y;
   const int b = blockIdx.z;
   const int head_coord = kShard ? b * H + h : h;  // head coordinate in the tensor maps
-  const int n_kv = (Skv + kBlockN - 1) / kBlockN;
+  const int n_kv_all = (Skv + kBlockN - 1) / kBlockN;
+  const int kv_base = n_kv_all / n_split, kv_rem = n_kv_all % n_split;
+  const int j0 = split * kv_base + (split < kv_rem ? split : kv_rem);  // first key block
+  const int n_kv = kv_base + (split < kv_rem ? 1 : 0);                 // key blocks here
+  if (n_split > 1) {
+    out = static_cast<char*>(out) + size_t(split) * gridDim.z * Sq * H * D * (kOutF32 ? 4 : 2);
+    lse += size_t(split) * gridDim.z * H * Sq;
+  }
   volatile int* abort_flag = &abort_sh;
 
   if (threadIdx.x == 0) {
@@ -180,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < kBlockN; ++c) x[c] = __uint_as_float(r[c]);
       }
-      const int valid = Skv - j * kBlockN;  // keys of this tile inside the sequence
+      const int valid = Skv - (j0 + j) * kBlockN;  // keys of this block inside the sequence
       if (valid < kBlockN) {
 #pragma unroll
         for (int c = 0; c < kBlockN; ++c)
@@ -401,7 +412,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t bar_f = smem_u32(&bars.full[slot]);
         mbar_arrive_expect_tx(bar_f, G::kTileBytes);
         load_tile((use & 1) ? &tm_v : &tm_k, (use & 1) ? &tm_v16 : &tm_k16,
-                  smem_base + G::kOffSlots + slot * G::kTileBytes, bar_f, (use >> 1) * kBlockN);
+                  smem_base + G::kOffSlots + slot * G::kTileBytes, bar_f,
+                  (j0 + (use >> 1)) * kBlockN);
         issued = use + 1;
       }
       // drain: every issued copy must have landed before the CTA's shared memory is
@@ -497,7 +509,7 @@ template <int D, bool kOutF32, int kMode>
 cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const CUtensorMap& tq16, const CUtensorMap& tk16, const CUtensorMap& tv16,
                    void* out, float* lse, dim3 grid, int H, int Sq, int Skv, float scale_log2,
-                   float rescale_log2, int s_local, int* err, long long wait_limit,
+                   float rescale_log2, int s_local, int n_split, int* err, long long wait_limit,
                    cudaStream_t stream) {
   using G = Geometry<D>;
   auto kernel = attn_fwd_sm100_kernel<D, kOutF32, kMode>;
@@ -505,8 +517,8 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
                                        G::kDynSmem);
   if (e != cudaSuccess) return e;
   kernel<<<grid, kThreads, G::kDynSmem, stream>>>(tq, tk, tv, tq16, tk16, tv16, out, lse, H, Sq,
-                                                   Skv, scale_log2, rescale_log2, s_local, err,
-                                                   wait_limit);
+                                                   Skv, scale_log2, rescale_log2, s_local, n_split,
+                                                   err, wait_limit);
   return cudaGetLastError();
 }
 
@@ -515,44 +527,49 @@ cudaError_t launch_o(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
                      const CUtensorMap& tq16, const CUtensorMap& tk16, const CUtensorMap& tv16,
                      void* out,
                      float* lse, dim3 grid, int H, int Sq, int Skv, float scale_log2,
-                     float rescale_log2, int s_local, bool out_f32, int* err, long long wait_limit,
-                     cudaStream_t stream) {
-  return out_f32 ? launch<D, true, kMode>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv, scale_log2,
-                                          rescale_log2, s_local, err, wait_limit, stream)
-                 : launch<D, false, kMode>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv, scale_log2,
-                                           rescale_log2, s_local, err, wait_limit, stream);
+                     float rescale_log2, int s_local, int n_split, bool out_f32, int* err,
+                     long long wait_limit, cudaStream_t stream) {
+  return out_f32 ? launch<D, true, kMode>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv,
+                                          scale_log2, rescale_log2, s_local, n_split, err,
+                                          wait_limit, stream)
+                 : launch<D, false, kMode>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv,
+                                           scale_log2, rescale_log2, s_local, n_split, err,
+                                           wait_limit, stream);
 }
 
 template <int D>
 cudaError_t launch_m(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      const CUtensorMap& tq16, const CUtensorMap& tk16, const CUtensorMap& tv16,
-                     void* out,
-                     float* lse, dim3 grid, int H, int Sq, int Skv, float scale_log2,
-                     float rescale_log2, int s_local, bool out_f32, int mode, int* err,
-                     long long wait_limit, cudaStream_t stream) {
+                     void* out, float* lse, dim3 grid, int H, int Sq, int Skv, float scale_log2,
+                     float rescale_log2, int s_local, int n_split, bool out_f32, int mode,
+                     int* err, long long wait_limit, cudaStream_t stream) {
   switch (mode) {
     case kAccum:
-      return launch_o<D, kAccum>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv, scale_log2, rescale_log2,
-                                 s_local, out_f32, err, wait_limit, stream);
+      return launch_o<D, kAccum>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv,
+                                 scale_log2, rescale_log2, s_local, n_split, out_f32, err,
+                                 wait_limit, stream);
     case kSharded:
-      return launch_o<D, kSharded>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv, scale_log2,
-                                   rescale_log2, s_local, out_f32, err, wait_limit, stream);
+      return launch_o<D, kSharded>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv,
+                                   scale_log2, rescale_log2, s_local, n_split, out_f32, err,
+                                   wait_limit, stream);
     default:
-      return launch_o<D, kPlain>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv, scale_log2, rescale_log2,
-                                 s_local, out_f32, err, wait_limit, stream);
+      return launch_o<D, kPlain>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv,
+                                 scale_log2, rescale_log2, s_local, n_split, out_f32, err,
+                                 wait_limit, stream);
   }
 }
 
 cudaError_t launch_any(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tq16, const CUtensorMap& tk16, const CUtensorMap& tv16,
                        void* out, float* lse, dim3 grid, int H, int Sq, int Skv, int D,
-                       float scale_log2, float rescale_log2, int s_local, bool out_f32, int mode,
-                       int* err, long long wait_limit, cudaStream_t stream) {
+                       float scale_log2, float rescale_log2, int s_local, int n_split,
+                       bool out_f32, int mode, int* err, long long wait_limit,
+                       cudaStream_t stream) {
   if (D == 128)
-    return launch_m<128>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv, scale_log2, rescale_log2, s_local,
-                         out_f32, mode, err, wait_limit, stream);
-  return launch_m<64>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv, scale_log2, rescale_log2, s_local,
-                      out_f32, mode, err, wait_limit, stream);
+    return launch_m<128>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv, scale_log2,
+                         rescale_log2, s_local, n_split, out_f32, mode, err, wait_limit, stream);
+  return launch_m<64>(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, H, Sq, Skv, scale_log2,
+                      rescale_log2, s_local, n_split, out_f32, mode, err, wait_limit, stream);
 }
 
 }  // namespace
@@ -560,25 +577,24 @@ cudaError_t launch_any(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
 cudaError_t launch_attn_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
                                   const CUtensorMap& tv, void* out, float* lse, int B, int H,
                                   int Sq, int Skv, int D, float scale_log2, float rescale_log2,
-                                  bool out_f32, bool accumulate, int* err, long long wait_limit,
-                                  cudaStream_t stream) {
-  const dim3 grid((Sq + 2 * kBlockM - 1) / (2 * kBlockM), H, B);
-  return launch_any(tq, tk, tv, tq, tk, tv, out, lse, grid, H, Sq, Skv, D, scale_log2, rescale_log2, 0,
-                    out_f32, accumulate ? kAccum : kPlain, err, wait_limit, stream);
+                                  bool out_f32, bool accumulate, int n_split, int* err,
+                                  long long wait_limit, cudaStream_t stream) {
+  const dim3 grid(((Sq + 2 * kBlockM - 1) / (2 * kBlockM)) * n_split, H, B);
+  return launch_any(tq, tk, tv, tq, tk, tv, out, lse, grid, H, Sq, Skv, D, scale_log2,
+                    rescale_log2, 0, n_split, out_f32, accumulate ? kAccum : kPlain, err,
+                    wait_limit, stream);
 }
 
 cudaError_t launch_ulysses_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
                                      const CUtensorMap& tv, const CUtensorMap& tq16,
                                      const CUtensorMap& tk16, const CUtensorMap& tv16, void* out,
-                                     float* lse, int P,
-                                     int S_local, int H, int D, float scale_log2,
-                                     float rescale_log2, bool out_f32, int* err,
+                                     float* lse, int P, int S_local, int H, int D,
+                                     float scale_log2, float rescale_log2, bool out_f32, int* err,
                                      long long wait_limit, cudaStream_t stream) {
   const int S = P * S_local, Hp = H / P;
   const dim3 grid((S + 2 * kBlockM - 1) / (2 * kBlockM), Hp, P);
   return launch_any(tq, tk, tv, tq16, tk16, tv16, out, lse, grid, Hp, S, S, D, scale_log2,
-                    rescale_log2, S_local,
-                    out_f32, kSharded, err, wait_limit, stream);
+                    rescale_log2, S_local, 1, out_f32, kSharded, err, wait_limit, stream);
 }
 
 }  // namespace cpattn

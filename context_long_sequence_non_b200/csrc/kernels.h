@@ -13,11 +13,14 @@ constexpr long long kDefaultWaitLimit = 2000000000LL;
 // tcgen05 attention, bf16 in, D in {64, 128}; tensor maps describe [B][S][H][D] bf16
 // tensors with a 64 x 1 x 128 x 1 box and 128-byte swizzle.  With `accumulate` the result
 // is merged into (out, lse) in place (the Ring Attention step) instead of overwriting it.
+// With n_split > 1 the key blocks are divided into n_split contiguous ranges, one CTA per
+// (query tile pair, range); range s writes its partial to out + s * B*Sq*H*D elements and
+// lse + s * B*H*Sq (combine them with launch_combine).
 cudaError_t launch_attn_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
                                   const CUtensorMap& tv, void* out, float* lse, int B, int H,
                                   int Sq, int Skv, int D, float scale_log2, float rescale_log2,
-                                  bool out_f32, bool accumulate, int* err, long long wait_limit,
-                                  cudaStream_t stream);
+                                  bool out_f32, bool accumulate, int n_split, int* err,
+                                  long long wait_limit, cudaStream_t stream);
 
 // Ulysses fused: q/k/v/out are [P][S_local][H][D] rank shards, each described by two tensor
 // maps over dims (D, H, S_local, P): a 64 x 1 x 128 x 1 box and a 64 x 1 x 16 x 1 box (for
@@ -47,6 +50,12 @@ cudaError_t launch_fill_empty(void* out, size_t out_bytes, float* lse, size_t n_
 cudaError_t launch_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
                          void* o, float* lse, int B, int H, int S, int D, int elem_bytes,
                          cudaStream_t stream);
+
+// Fold n (1..8) split-KV partials [n][B][S][H][D] (elem_bytes dtype) + LSE [n][B][H][S]
+// into (out, lse); with `accumulate` the running (out, lse) is one more term.
+cudaError_t launch_combine(const void* part_o, const float* part_lse, int n, void* out, float* lse,
+                           int B, int H, int S, int D, int elem_bytes, bool accumulate,
+                           cudaStream_t stream);
 
 // Ulysses permutes over 16-byte words; `run_vec` = Hp*D*elem_bytes/16.
 cudaError_t launch_seq2head(const void* src, void* dst, int P, int S_local, long long run_vec,

@@ -160,6 +160,86 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
   if (live && v == 0) lse[li] = L;
 }
 
+// ------------------------------------------------------------------ split-KV combine
+// n partial results of the same queries over disjoint key ranges (split-KV), each a
+// normalised O (dtype of out) with its LSE, are folded exactly -- optionally together with
+// the running accumulator already in (out, lse) -- by the same merge formula generalised to
+// n terms: L = max_s L_s + ln sum_s exp(L_s - max), O = sum_s exp(L_s - L) O_s.  Thread
+// layout as the merge kernel: one 16-byte vector of the row per thread, whole rows per block,
+// the output LSE written after a block barrier.
+constexpr int kMaxSplit = 8;
+
+template <bool kBf16, bool kAcc>
+__global__ void __launch_bounds__(kMergeThreads) combine_kernel(
+    const uint4* __restrict__ part_o, const float* __restrict__ part_lse, int n,
+    long long o_stride, long long lse_stride, uint4* out, float* lse, int H, int S,
+    long long n_rows, int vpr) {
+  const int rows_per_block = blockDim.x / vpr;
+  const int rl = threadIdx.x / vpr;
+  const int v = threadIdx.x - rl * vpr;
+  const long long row = (long long)blockIdx.x * rows_per_block + rl;  // (b, s, h), h fastest
+  const bool live = row < n_rows;
+  long long li = 0;
+  float L = -INFINITY;
+  if (live) {
+    const int h = int(row % H);
+    const long long bs = row / H;
+    const int si = int(bs % S);
+    const long long b = bs / S;
+    li = (b * H + h) * S + si;
+    const long long idx = row * vpr + v;
+    float ls[kMaxSplit + 1];
+    float mx = -INFINITY;
+    for (int t = 0; t < n; ++t) {
+      ls[t] = part_lse[t * lse_stride + li];
+      mx = fmaxf(mx, ls[t]);
+    }
+    const float la = kAcc ? lse[li] : -INFINITY;
+    mx = fmaxf(mx, la);
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    float tot = 0.f;
+    if (mx != -INFINITY) {
+      for (int t = 0; t <= n; ++t) {
+        const float lt = t < n ? ls[t] : la;
+        if (lt == -INFINITY) continue;  // an empty term contributes nothing (and is not read)
+        const float wgt = expf(lt - mx);
+        tot += wgt;
+        const uint4 p = t < n ? part_o[t * o_stride + idx] : out[idx];
+        if (kBf16) {
+          const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            acc[2 * e] = fmaf(wgt, __uint_as_float(pw[e] << 16), acc[2 * e]);
+            acc[2 * e + 1] = fmaf(wgt, __uint_as_float(pw[e] & 0xFFFF0000u), acc[2 * e + 1]);
+          }
+        } else {
+          acc[0] = fmaf(wgt, __uint_as_float(p.x), acc[0]);
+          acc[1] = fmaf(wgt, __uint_as_float(p.y), acc[1]);
+          acc[2] = fmaf(wgt, __uint_as_float(p.z), acc[2]);
+          acc[3] = fmaf(wgt, __uint_as_float(p.w), acc[3]);
+        }
+      }
+      L = mx + logf(tot);
+    }
+    const float inv = tot > 0.f ? 1.0f / tot : 0.f;
+    uint4 r;
+    if (kBf16) {
+      r.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+      r.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+      r.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+      r.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+    } else {
+      r = make_uint4(__float_as_uint(acc[0] * inv), __float_as_uint(acc[1] * inv),
+                     __float_as_uint(acc[2] * inv), __float_as_uint(acc[3] * inv));
+    }
+    out[idx] = r;
+  }
+  __syncthreads();
+  if (live && v == 0 && lse != nullptr) lse[li] = L;
+}
+
 // ------------------------------------------------------------------ Ulysses permutes
 // Rows of Hp*D elements move as whole 16-byte-vector runs.  Head-grouped row index
 // A(g, r, s) = (g*P + r)*S_l + s; sequence-sharded row index Bq(g, r, s) = (r*S_l + s)*P + g.
@@ -324,6 +404,35 @@ cudaError_t launch_merge(const void* o_a, const float* lse_a, const void* o_b, c
     merge_kernel<false><<<unsigned(blocks), threads, 0, stream>>>(
         static_cast<const uint4*>(o_a), lse_a, static_cast<const uint4*>(o_b), lse_b,
         static_cast<uint4*>(o), lse, H, S, n_rows, vpr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const void* part_o, const float* part_lse, int n, void* out, float* lse,
+                           int B, int H, int S, int D, int elem_bytes, bool accumulate,
+                           cudaStream_t stream) {
+  if (n < 1 || n > kMaxSplit) return cudaErrorInvalidValue;
+  const long long n_rows = (long long)B * S * H;
+  const int vpr = D * elem_bytes / 16;
+  const int rows_per_block = vpr >= kMergeThreads ? 1 : kMergeThreads / vpr;
+  const long long blocks = (n_rows + rows_per_block - 1) / rows_per_block;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  const int threads = rows_per_block * vpr;
+  const long long o_stride = n_rows * vpr;  // 16-byte vectors per partial
+  const long long lse_stride = (long long)B * H * S;
+  const uint4* po = static_cast<const uint4*>(part_o);
+  uint4* o = static_cast<uint4*>(out);
+#define CPATTN_COMBINE(BF, ACC)                                                             \
+  combine_kernel<BF, ACC><<<unsigned(blocks), threads, 0, stream>>>(po, part_lse, n, o_stride, \
+                                                                    lse_stride, o, lse, H, S,   \
+                                                                    n_rows, vpr)
+  if (elem_bytes == 2) {
+    if (accumulate) CPATTN_COMBINE(true, true);
+    else CPATTN_COMBINE(true, false);
+  } else {
+    if (accumulate) CPATTN_COMBINE(false, true);
+    else CPATTN_COMBINE(false, false);
+  }
+#undef CPATTN_COMBINE
   return cudaGetLastError();
 }
 

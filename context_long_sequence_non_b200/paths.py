@@ -19,14 +19,17 @@ import torch
 from . import _binding as B
 
 
-def ring_attention(q, k_chunks, v_chunks, scale=None, acc_dtype=None, fused=True, stream=None):
+def ring_attention(q, k_chunks, v_chunks, scale=None, acc_dtype=None, fused=True, n_split=1,
+                   stream=None):
     """One rank's ring step over K/V chunks in ring order.
 
     q: [B][Sq][H][D]; each chunk [B][S_c][H][D].  The running (O, LSE) is kept in
     ``acc_dtype`` (default: q's dtype).  ``fused=True`` (default) merges every chunk into
     the accumulator inside the attention epilogue (cpattn_fwd_accumulate); ``fused=False``
-    writes each chunk's partial and folds it with the separate merge kernel.  Returns
-    ``(O, LSE)``.
+    writes each chunk's partial and folds it with the separate merge kernel.  With the fused
+    form, ``n_split`` > 1 (or None: the library's suggestion) computes every chunk as that
+    many key ranges folded straight into the accumulator (split-KV, for query slices too
+    small to fill the GPU).  Returns ``(O, LSE)``.
     """
     if scale is None:
         scale = 1.0 / math.sqrt(q.shape[3])
@@ -35,6 +38,16 @@ def ring_attention(q, k_chunks, v_chunks, scale=None, acc_dtype=None, fused=True
     acc_o = torch.empty((Bn, Sq, H, D), dtype=acc_dtype, device=q.device)
     acc_l = torch.empty((Bn, H, Sq), dtype=torch.float32, device=q.device)
     if fused:
+        if n_split is None:
+            n_split = B.split_suggest(Bn, H, Sq, k_chunks[0].shape[1])
+        if n_split > 1:
+            ws = torch.empty(max(B.split_workspace_bytes(Bn, H, Sq, D, n_split, acc_dtype), 256),
+                             dtype=torch.uint8, device=q.device)
+            acc_l.fill_(-math.inf)  # empty accumulator: its O rows are never read
+            for kc, vc in zip(k_chunks, v_chunks):
+                B.fwd_split(q, kc, vc, out=acc_o, lse=acc_l, scale=scale, accumulate=True,
+                            n_split=n_split, workspace=ws, stream=stream)
+            return acc_o, acc_l
         for c, (kc, vc) in enumerate(zip(k_chunks, v_chunks)):
             if c == 0:
                 B.fwd(q, kc, vc, out=acc_o, lse=acc_l, scale=scale, stream=stream)

@@ -29,6 +29,8 @@
 #ifndef CPATTN_H
 #define CPATTN_H
 
+#include <stddef.h>
+
 #if defined(__GNUC__)
 #define CPATTN_API __attribute__((visibility("default")))
 #else
@@ -85,6 +87,38 @@ typedef enum {
 CPATTN_API int cpattn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
                int B, int H, int Sq, int Skv, int D, float scale,
                int in_dtype, int out_dtype, cpattn_stream_t stream);
+
+/*
+ * cpattn_fwd_split -- cpattn_fwd (accumulate = 0) or cpattn_fwd_accumulate (accumulate = 1)
+ * computed as n_split independent key ranges ("split-KV") whose partial (O, LSE) results
+ * are then folded exactly by the merge formula of the Ring Attention step (Fig. 3) --
+ * the online softmax makes partials over disjoint key sets combine losslessly.  It exists
+ * for shapes with too few (query tile, head) work items to fill the GPU, e.g. one rank's
+ * 5520-token query slice against a K/V chunk: 352 CTAs are 2.4 waves on 148 SMs, while
+ * two key ranges give 704 CTAs.  Same arguments and results as the single-pass calls
+ * (bf16 inputs, D in {64, 128}); with n_split = 1 it is exactly that call.
+ * workspace : caller-owned device buffer, 256-byte aligned, of at least
+ *   cpattn_fwd_split_workspace(B, H, Sq, D, n_split, out_dtype) bytes; it receives the
+ *   partials ([n_split][B][Sq][H][D] in out_dtype, then [n_split][B][H][Sq] float32).
+ *   Concurrent calls must not share it.
+ * Errors: as cpattn_fwd / cpattn_fwd_accumulate; CPATTN_ERR_SHAPE for n_split outside 1..8
+ *   or a workspace that is too small; CPATTN_ERR_ALIGN for its alignment.
+ */
+CPATTN_API int cpattn_fwd_split(const void* q, const void* k, const void* v, void* out, float* lse,
+                                int B, int H, int Sq, int Skv, int D, float scale, int out_dtype,
+                                int accumulate, int n_split, void* workspace,
+                                size_t workspace_bytes, cpattn_stream_t stream);
+
+/* Workspace bytes cpattn_fwd_split needs (0 for n_split = 1 or invalid sizes). */
+CPATTN_API size_t cpattn_fwd_split_workspace(int B, int H, int Sq, int D, int n_split,
+                                             int out_dtype);
+
+/*
+ * cpattn_split_suggest -- split count (1..8) the library's wave model prefers for this
+ * shape on the current device: 1 when the (query tile pair, head) grid already fills the
+ * SMs for four or more waves.
+ */
+CPATTN_API int cpattn_split_suggest(int B, int H, int Sq, int Skv);
 
 /*
  * cpattn_ulysses_fwd -- the whole DeepSpeed Ulysses attention of one layer in one kernel

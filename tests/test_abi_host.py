@@ -101,6 +101,34 @@ def test_ulysses_fwd_argument_errors(L):
     assert uf(q=FAKE + 8) == B.ERR_ALIGN
 
 
+def test_fwd_split_argument_errors_and_sizes(L):
+    vp = ctypes.c_void_p
+
+    def fs(n=2, ws=FAKE, ws_bytes=1 << 30, lse=FAKE, acc=0, D=128):
+        return L.cpattn_fwd_split(vp(FAKE), vp(FAKE), vp(FAKE), vp(FAKE), vp(lse) if lse else None,
+                                  1, 2, 512, 4096, D, 0.1, 0, acc, n, vp(ws) if ws else None,
+                                  ws_bytes, None)
+
+    assert fs(n=9) == B.ERR_SHAPE
+    assert fs(n=0) == B.ERR_SHAPE
+    assert fs(ws=0) == B.ERR_NULL
+    assert fs(ws=FAKE + 16) == B.ERR_ALIGN  # 256-byte alignment
+    assert fs(ws_bytes=1000) == B.ERR_SHAPE  # too small
+    assert fs(lse=0, acc=1) == B.ERR_NULL
+    assert fs(D=96) == B.ERR_UNSUPPORTED
+    need = L.cpattn_fwd_split_workspace(1, 2, 512, 128, 2, 0)
+    assert need == 2 * 512 * 2 * 128 * 2 + 2 * 2 * 512 * 4
+    assert L.cpattn_fwd_split_workspace(1, 2, 512, 128, 1, 0) == 0
+    assert L.cpattn_fwd_split_workspace(1, 2, 512, 128, 9, 0) == 0
+
+
+def test_split_suggestion_model():
+    assert B.split_suggest(8, 2, 44160, 44160) == 1  # 2768 CTAs: many waves already
+    assert B.split_suggest(1, 16, 512, 44160) >= 4   # 32 CTAs over 345 key blocks: split
+    assert B.split_suggest(1, 16, 5520, 5520) == 1   # 352 CTAs of 43 blocks: start-up eats it
+    assert B.split_suggest(1, 1, 128, 128) == 1       # too few key blocks to split
+
+
 def test_merge_argument_errors(L):
     vp = ctypes.c_void_p
     base = [vp(FAKE), vp(FAKE + 0x100000), vp(FAKE + 0x200000), vp(FAKE + 0x300000),

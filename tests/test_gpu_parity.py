@@ -218,6 +218,50 @@ def test_fused_ring_accumulate_matches_oracle(shape, split, acc):
         assert (o_acc - om).abs().max().item() < 1e-5
 
 
+@pytest.mark.parametrize("shape,n_split", [((1, 2, 300, 1000, 128), 2), ((1, 1, 129, 129, 64), 3),
+                                           ((2, 3, 200, 1100, 128), 8), ((1, 4, 70, 600, 128), 4)])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_split_kv_matches_single_pass_and_oracle(shape, n_split, out_dtype):
+    Bn, H, Sq, Skv, D = shape
+    q, k, v = W.random_case(Sq * 3 + n_split, Bn, H, Sq, Skv, D)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    o_s, l_s = cp.fwd_split(qd, kd, vd, out_dtype=out_dtype, n_split=n_split)
+    o_1, l_1 = cp.fwd(qd, kd, vd, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    o_ref, l_ref = ref.attention(q, k, v, 1 / math.sqrt(D))
+    kind = "bf16_out" if out_dtype == torch.bfloat16 else "bf16_in"
+    check_o(o_s, o_ref, kind, f"split {n_split}")
+    check_lse(l_s, l_ref, f"split {n_split}")
+    assert (l_s - l_1).abs().max().item() < 2e-5
+    if out_dtype == torch.float32:
+        # each key range subtracts its own row max before P is rounded to bf16, so the
+        # two forms differ at the level of bf16 P rounding, not beyond
+        assert (o_s - o_1).abs().max().item() < 2e-3
+    # accumulate: a second pass over the same keys adds ln 2 and keeps O
+    o_a, l_a = o_s.clone(), l_s.clone()
+    cp.fwd_split(qd, kd, vd, out=o_a, lse=l_a, accumulate=True, n_split=n_split)
+    torch.cuda.synchronize()
+    assert ((l_a - l_s) - math.log(2)).abs().max().item() < 2e-5
+    tol = 2e-5 if out_dtype == torch.float32 else 1e-2
+    assert (o_a.float() - o_s.float()).abs().max().item() < tol
+
+
+def test_ring_step_with_split_kv():
+    w = W.WORKLOADS[3]
+    x = W.make_inputs(w)
+    q, k, v = (x[n].to(DEV) for n in ("q", "k", "v"))
+    c = x["chunks"][0]
+    kc = [k[:, i * c:(i + 1) * c].contiguous() for i in range(len(x["chunks"]))]
+    vc = [v[:, i * c:(i + 1) * c].contiguous() for i in range(len(x["chunks"]))]
+    o_s, l_s = cp.ring_attention(q, kc, vc, acc_dtype=torch.float32, n_split=2)
+    o_1, l_1 = cp.ring_attention(q, kc, vc, acc_dtype=torch.float32, n_split=1)
+    torch.cuda.synchronize()
+    assert (o_s - o_1).abs().max().item() < 2e-3 and (l_s - l_1).abs().max().item() < 2e-5
+    rows = W.sample_rows(w.B, w.H, w.Sq, 512, seed=33)
+    _sampled(x["q"], x["k"], x["v"], w.softmax_scale, o_s.cpu(), l_s.cpu(), rows, "bf16_in",
+             "ring split-KV")
+
+
 def test_accumulate_empty_chunk_is_identity():
     q, k, v = (t.to(DEV) for t in W.random_case(3, 1, 2, 40, 50, 128))
     o, l = cp.fwd(q, k, v, out_dtype=torch.float32)
