@@ -121,6 +121,35 @@ CPATTN_API size_t cpattn_fwd_split_workspace(int B, int H, int Sq, int D, int n_
 CPATTN_API int cpattn_split_suggest(int B, int H, int Sq, int Skv);
 
 /*
+ * cpattn_fwd_split_noalloc -- cpattn_fwd_split for callers that cannot allocate device
+ * memory: code running inside a host runtime that owns all device memory and hands out no
+ * workspace (an inference-engine plugin, for instance), or a latency-critical loop that
+ * must not call cudaMalloc/cudaFree, which can synchronize the whole device.  The pages
+ * have no counterpart to this call; it is a library convenience.
+ * Same arguments and results as cpattn_fwd_split without the workspace arguments: the
+ * partials go to a fixed scratch array compiled into the library,
+ * cpattn_noalloc_scratch_bytes() = 64 MiB, which every GPU that loads the library holds
+ * until the process exits.  The call itself allocates nothing: it makes no cudaMalloc,
+ * cudaFree or other allocating call.
+ * The first call on a device looks up that device's address of the array (with the device
+ * current); make that first call before any stream capture.
+ * All calls on a device share the one array and it keeps the last call's contents (each
+ * call writes every byte it reads first, so nothing needs clearing): calls that overlap on
+ * the GPU -- on different streams, or from different threads -- race on it and must not
+ * be issued.
+ * Errors: as cpattn_fwd_split; CPATTN_ERR_SHAPE also when the partials need more than
+ *   cpattn_noalloc_scratch_bytes() (cpattn_fwd_split_workspace(B, H, Sq, D, n_split,
+ *   out_dtype) tells), checked before anything is launched.
+ */
+CPATTN_API int cpattn_fwd_split_noalloc(const void* q, const void* k, const void* v, void* out,
+                                        float* lse, int B, int H, int Sq, int Skv, int D,
+                                        float scale, int out_dtype, int accumulate, int n_split,
+                                        cpattn_stream_t stream);
+
+/* Size in bytes of the fixed scratch behind cpattn_fwd_split_noalloc (64 MiB). */
+CPATTN_API size_t cpattn_noalloc_scratch_bytes(void);
+
+/*
  * cpattn_ulysses_fwd -- the whole DeepSpeed Ulysses attention of one layer in one kernel
  * (Fig. 4: all-to-all from sequence shards to head groups, full-sequence attention per head
  * group, all-to-all back), for P virtual ranks on one GPU.  The result equals
