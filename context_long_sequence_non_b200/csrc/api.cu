@@ -230,6 +230,7 @@ int cpattn_fwd_split(const void* q, const void* k, const void* v, void* out, flo
       !aligned(workspace, 256) || (lse != nullptr && !aligned(lse, 4)))
     return CPATTN_ERR_ALIGN;
   if (workspace_bytes < split_ws_bytes(B, H, Sq, D, n_split, es)) return CPATTN_ERR_SHAPE;
+  if ((long long)B * Sq * H > 0x7fffffffLL) return CPATTN_ERR_SHAPE;  // 32-bit row index
   int* err = device_error_word();
   if (err == nullptr) return CPATTN_ERR_CUDA;
   CUtensorMap tq, tk, tv;
@@ -285,6 +286,7 @@ int cpattn_merge(const void* o_a, const float* lse_a, const void* o_b, const flo
   const int es = elem_size(dtype);
   if (es == 0) return CPATTN_ERR_UNSUPPORTED;
   if ((D * es) % 16 != 0 || D * es > 4096) return CPATTN_ERR_SHAPE;
+  if ((long long)B * S * H > 0x7fffffffLL - 4096) return CPATTN_ERR_SHAPE;  // 32-bit row index
   if (!o_a || !lse_a || !o_b || !lse_b || !o || !lse) return CPATTN_ERR_NULL;
   if (!aligned(o_a, 16) || !aligned(o_b, 16) || !aligned(o, 16) || !aligned(lse_a, 4) ||
       !aligned(lse_b, 4) || !aligned(lse, 4))
@@ -305,7 +307,8 @@ static int permute_args(const void* src, void* dst, int P, int S_local, int H, i
   if (H % P != 0) return CPATTN_ERR_SHAPE;
   const long long run_bytes = (long long)(H / P) * D * elem_bytes;
   if (run_bytes % 16 != 0) return CPATTN_ERR_SHAPE;
-  if ((long long)P * P * S_local > 0x7fffffffLL || run_bytes / 16 > 0x7fffffffLL)
+  // item indices are 32-bit: rows x 32-vector chunks must stay below 2^31
+  if ((long long)P * P * S_local * ((run_bytes / 16 + 31) / 32) > 0x7fffffffLL)
     return CPATTN_ERR_SHAPE;
   if (src == nullptr || dst == nullptr) return CPATTN_ERR_NULL;
   if (!aligned(src, 16) || !aligned(dst, 16)) return CPATTN_ERR_ALIGN;

@@ -92,9 +92,10 @@ __global__ void fill_empty_kernel(uint4* out, size_t n_vec, float* lse, size_t n
 }
 
 // ------------------------------------------------------------------ (O, LSE) merge
-// One 16-byte vector of O per thread; a block covers whole (b, s, h) rows (blockDim =
-// rows_per_block x vectors_per_row).  Every thread derives its row's weights from the two
-// LSEs itself (no shared-memory phase), so loads of O and LSE are all in flight at once.
+// 16-byte vectors of O; a block covers whole (b, s, h) rows (blockDim = rows x
+// vectors_per_row) and every thread handles kMergeRowsPerThread rows.  Every thread derives
+// its rows' weights from the two LSEs itself (no shared-memory phase), so the loads of O and
+// LSE for all its rows are in flight at once.
 // The merged LSE is written after a block barrier by the row's first thread: every read of
 // this block's LSE entries precedes every write, and each O vector is read and written by
 // the same thread, so the result may overwrite partial a in place.
@@ -121,43 +122,65 @@ __device__ __forceinline__ void merge_vec_f32(const uint4& a, const uint4& b, fl
   o.w = __float_as_uint(fmaf(wa, __uint_as_float(a.w), wb * __uint_as_float(b.w)));
 }
 
+constexpr int kMergeRowsPerThread = 4;  // independent row vectors in flight per thread
+
 template <bool kBf16>
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
     const uint4* o_a, const float* lse_a, const uint4* o_b, const float* lse_b, uint4* o,
     float* lse, int H, int S, long long n_rows, int vpr) {
-  const int rows_per_block = blockDim.x / vpr;
+  // a block covers kMergeRowsPerThread groups of (blockDim.x / vpr) consecutive rows; thread
+  // (rl, v) takes vector v of row rl of every group, issuing all loads before any math
+  const int rows_per_group = blockDim.x / vpr;
   const int rl = threadIdx.x / vpr;
   const int v = threadIdx.x - rl * vpr;
-  const long long row = (long long)blockIdx.x * rows_per_block + rl;  // (b, s, h), h fastest
-  const bool live = rl < rows_per_block && row < n_rows;
-  long long li = 0;
-  float L = -INFINITY;
-  if (live) {
-    const int h = int(row % H);
-    const long long bs = row / H;
-    const int s = int(bs % S);
-    const long long b = bs / S;
-    li = (b * H + h) * S + s;
-    const long long idx = row * vpr + v;
-    const uint4 a = o_a[idx];
-    const uint4 bv = o_b[idx];
-    const float la = lse_a[li], lb = lse_b[li];
-    const float mx = fmaxf(la, lb);
+  const int row0 = int(blockIdx.x) * rows_per_group * kMergeRowsPerThread + rl;
+  uint4 a[kMergeRowsPerThread], bb[kMergeRowsPerThread];
+  float la[kMergeRowsPerThread], lb[kMergeRowsPerThread];
+  int li[kMergeRowsPerThread];
+  bool live[kMergeRowsPerThread];
+#pragma unroll
+  for (int u = 0; u < kMergeRowsPerThread; ++u) {
+    const int row = row0 + u * rows_per_group;  // (b, s, h), h fastest; < 2^31
+    live[u] = row < n_rows;
+    const int bs = row / H;
+    const int h = row - bs * H;
+    const int b = bs / S;
+    const int s = bs - b * S;
+    li[u] = (b * H + h) * S + s;
+    if (live[u]) {
+      const long long idx = (long long)row * vpr + v;
+      a[u] = o_a[idx];
+      bb[u] = o_b[idx];
+      la[u] = lse_a[li[u]];
+      lb[u] = lse_b[li[u]];
+    }
+  }
+  float L[kMergeRowsPerThread];
+#pragma unroll
+  for (int u = 0; u < kMergeRowsPerThread; ++u) {
+    L[u] = -INFINITY;
+    if (!live[u]) continue;
+    const float mx = fmaxf(la[u], lb[u]);
     float wa = 0.f, wb = 0.f;
     if (mx != -INFINITY) {
-      const float ea = expf(la - mx), eb = expf(lb - mx);
+      const float ea = expf(la[u] - mx), eb = expf(lb[u] - mx);
       const float tot = ea + eb;
-      L = mx + logf(tot);
+      L[u] = mx + logf(tot);
       wa = ea / tot;
       wb = eb / tot;
     }
     uint4 r;
-    if (kBf16) merge_vec_bf16(a, bv, wa, wb, r);
-    else merge_vec_f32(a, bv, wa, wb, r);
-    o[idx] = r;
+    if (kBf16) merge_vec_bf16(a[u], bb[u], wa, wb, r);
+    else merge_vec_f32(a[u], bb[u], wa, wb, r);
+    o[(long long)(row0 + u * rows_per_group) * vpr + v] = r;
   }
+  // every read of this block's LSE entries precedes every write (in-place merge allowed)
   __syncthreads();
-  if (live && v == 0) lse[li] = L;
+  if (v == 0) {
+#pragma unroll
+    for (int u = 0; u < kMergeRowsPerThread; ++u)
+      if (live[u]) lse[li[u]] = L[u];
+  }
 }
 
 // ------------------------------------------------------------------ split-KV combine
@@ -177,17 +200,17 @@ __global__ void __launch_bounds__(kMergeThreads) combine_kernel(
   const int rows_per_block = blockDim.x / vpr;
   const int rl = threadIdx.x / vpr;
   const int v = threadIdx.x - rl * vpr;
-  const long long row = (long long)blockIdx.x * rows_per_block + rl;  // (b, s, h), h fastest
+  const int row = int(blockIdx.x) * rows_per_block + rl;  // (b, s, h), h fastest; < 2^31
   const bool live = row < n_rows;
-  long long li = 0;
+  int li = 0;
   float L = -INFINITY;
   if (live) {
-    const int h = int(row % H);
-    const long long bs = row / H;
-    const int si = int(bs % S);
-    const long long b = bs / S;
+    const int bs = row / H;
+    const int h = row - bs * H;
+    const int b = bs / S;
+    const int si = bs - b * S;
     li = (b * H + h) * S + si;
-    const long long idx = row * vpr + v;
+    const long long idx = (long long)row * vpr + v;
     float ls[kMaxSplit + 1];
     float mx = -INFINITY;
     for (int t = 0; t < n; ++t) {
@@ -256,46 +279,44 @@ struct PermuteSet {
 
 template <bool kToHead>
 __global__ void __launch_bounds__(kPermThreads) permute_kernel(const __grid_constant__ PermuteSet set,
-                                                                int n_tensors, int P, int S_l,
-                                                                int run_vec, int chunks,
-                                                                long long n_items) {
+                                                                int P, int S_l, int run_vec,
+                                                                int chunks, int n_items) {
+  // blockIdx.y picks the tensor (uniform per block); item = (dst row, 32-vector chunk)
+  const uint4* __restrict__ src = set.src[blockIdx.y];
+  uint4* __restrict__ dst = set.dst[blockIdx.y];
   const int lane = threadIdx.x & 31;
-  const long long warp = ((long long)blockIdx.x * kPermThreads + threadIdx.x) >> 5;
-  const long long n_warps = ((long long)gridDim.x * kPermThreads) >> 5;
-  const long long total = n_items * n_tensors;
-  for (long long it0 = warp * kPermUnroll; it0 < total; it0 += n_warps * kPermUnroll) {
+  const int warp = int((blockIdx.x * kPermThreads + threadIdx.x) >> 5);
+  const int n_warps = int((gridDim.x * kPermThreads) >> 5);
+  for (int it0 = warp * kPermUnroll; it0 < n_items; it0 += n_warps * kPermUnroll) {
     uint4 buf[kPermUnroll];
-    uint4* dst_ptr[kPermUnroll];
+    long long dst_off[kPermUnroll];
     bool live[kPermUnroll];
 #pragma unroll
     for (int u = 0; u < kPermUnroll; ++u) {
-      const long long itg = it0 + u;
-      const int tsel = int(itg / n_items);  // which tensor
-      const long long it = itg - (long long)tsel * n_items;
-      const long long n = it / chunks;  // dst row
-      const int v = int(it - n * chunks) * 32 + lane;
-      live[u] = itg < total && v < run_vec;
-      long long src_row = 0;
+      const int it = it0 + u;
+      const int n = it / chunks;  // dst row
+      const int v = (it - n * chunks) * 32 + lane;
+      live[u] = it < n_items && v < run_vec;
+      int src_row;
       if (kToHead) {  // n = A(g, r, s)
-        const int s = int(n % S_l);
-        const long long gr = n / S_l;
-        const int r = int(gr % P);
-        const int g = int(gr / P);
-        src_row = ((long long)r * S_l + s) * P + g;
+        const int gr = n / S_l;
+        const int s = n - gr * S_l;
+        const int g = gr / P;
+        const int r = gr - g * P;
+        src_row = (r * S_l + s) * P + g;
       } else {  // n = Bq(g, r, s)
-        const int g = int(n % P);
-        const long long rs = n / P;
-        const int s = int(rs % S_l);
-        const int r = int(rs / S_l);
-        src_row = ((long long)g * P + r) * S_l + s;
+        const int rs = n / P;
+        const int g = n - rs * P;
+        const int r = rs / S_l;
+        const int s = rs - r * S_l;
+        src_row = (g * P + r) * S_l + s;
       }
-      const int ts = live[u] ? tsel : 0;
-      dst_ptr[u] = set.dst[ts] + n * run_vec + v;
-      if (live[u]) buf[u] = set.src[ts][src_row * run_vec + v];
+      dst_off[u] = (long long)n * run_vec + v;
+      if (live[u]) buf[u] = src[(long long)src_row * run_vec + v];
     }
 #pragma unroll
     for (int u = 0; u < kPermUnroll; ++u)
-      if (live[u]) *dst_ptr[u] = buf[u];
+      if (live[u]) dst[dst_off[u]] = buf[u];
   }
 }
 
@@ -392,10 +413,11 @@ cudaError_t launch_merge(const void* o_a, const float* lse_a, const void* o_b, c
                          cudaStream_t stream) {
   const long long n_rows = (long long)B * S * H;
   const int vpr = D * elem_bytes / 16;  // 16-byte vectors per row (validated: 1..256)
-  const int rows_per_block = vpr >= kMergeThreads ? 1 : kMergeThreads / vpr;
+  const int rows_per_group = vpr >= kMergeThreads ? 1 : kMergeThreads / vpr;
+  const long long rows_per_block = (long long)rows_per_group * kMergeRowsPerThread;
   const long long blocks = (n_rows + rows_per_block - 1) / rows_per_block;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  const int threads = rows_per_block * vpr;
+  const int threads = rows_per_group * vpr;
   if (elem_bytes == 2)
     merge_kernel<true><<<unsigned(blocks), threads, 0, stream>>>(
         static_cast<const uint4*>(o_a), lse_a, static_cast<const uint4*>(o_b), lse_b,
@@ -448,16 +470,18 @@ static cudaError_t launch_permute(bool to_head, const void* const* src, void* co
   const long long n_rows = (long long)P * P * S_local;
   const int chunks = int((run_vec + 31) / 32);
   const long long n_items = n_rows * chunks;
-  const long long warps_needed = (n_items * n_tensors + kPermUnroll - 1) / kPermUnroll;
+  if (n_items > 0x7fffffffLL) return cudaErrorInvalidValue;  // 32-bit item index
+  const long long warps_needed = (n_items + kPermUnroll - 1) / kPermUnroll;
   const long long blocks_needed = (warps_needed * 32 + kPermThreads - 1) / kPermThreads;
-  const long long cap = (long long)sm_count() * 8;
+  const long long cap = (long long)sm_count() * 8 / n_tensors + 1;
   const long long blocks = blocks_needed < cap ? blocks_needed : cap;
+  const dim3 grid{unsigned(blocks), unsigned(n_tensors), 1u};
   if (to_head)
-    permute_kernel<true><<<unsigned(blocks), kPermThreads, 0, stream>>>(
-        set, n_tensors, P, S_local, int(run_vec), chunks, n_items);
+    permute_kernel<true><<<grid, kPermThreads, 0, stream>>>(set, P, S_local, int(run_vec), chunks,
+                                                            int(n_items));
   else
-    permute_kernel<false><<<unsigned(blocks), kPermThreads, 0, stream>>>(
-        set, n_tensors, P, S_local, int(run_vec), chunks, n_items);
+    permute_kernel<false><<<grid, kPermThreads, 0, stream>>>(set, P, S_local, int(run_vec), chunks,
+                                                             int(n_items));
   return cudaGetLastError();
 }
 

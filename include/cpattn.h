@@ -201,7 +201,7 @@ CPATTN_API int cpattn_fwd_accumulate(const void* q, const void* k, const void* v
  * lse_a, lse_b, lse : [B][H][S] float32.
  * o may alias o_a and lse may alias lse_a (in-place accumulate); no other overlap.
  * D must be a multiple of 8 (BF16) or 4 (F32) so rows move as 16-byte vectors, and a
- * row must fit in 4096 bytes (D <= 2048 BF16, 1024 F32).
+ * row must fit in 4096 bytes (D <= 2048 BF16, 1024 F32); B*S*H < 2^31.
  * Errors: CPATTN_ERR_NULL, _SHAPE, _ALIGN, _UNSUPPORTED (dtype), _CUDA.
  */
 CPATTN_API int cpattn_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
