@@ -37,6 +37,10 @@ from context_long_sequence_non_b200 import workloads as W  # noqa: E402
 METRIC = "non-causal bf16 attention TFLOPS at S=44160 on 1 B200; % of dense BF16 peak"
 UNIT = "TFLOP/s"
 WORKLOAD = W.WORKLOADS[4]
+# DRAM bytes (read + write) per launch of the attention kernel on this workload, from the
+# ncu capture summarised in profiles/attn_fwd_sm100_ulysses_s44160.md; valid only for the
+# kernel version named there (set to None whenever the kernel changes until re-captured).
+ATTN_TRAFFIC_BYTES = 580_206_336 + 172_326_912
 L2_NOTE = ("inputs larger than L2: each step streams 543 MB of Q/K/V shards plus 724 MB of "
            "permute traffic through the 126 MB L2")
 
@@ -254,7 +258,11 @@ def run_ours(args, world, rank, local):
             "peak_kind": (f"{peaks['source']} cuBLAS bf16 "
                           f"{'sustained' if long_run else 'burst'}"),
             "algorithmic_flops_per_launch": flops,
-            "avg_launch_ms": round(attn_ms, 4), "traffic": None,
+            "avg_launch_ms": round(attn_ms, 4), "traffic": ATTN_TRAFFIC_BYTES,
+            "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
+            # Q, K, V read once and O written once (four equal bf16 tensors) + fp32 LSE
+            "algorithmic_bytes_per_launch": 4 * q.numel() * q.element_size()
+            + plan.lse.numel() * 4,
         },
         "aux": aux,
         "e2e": e2e,
