@@ -40,7 +40,7 @@ WORKLOAD = W.WORKLOADS[4]
 # DRAM bytes (read + write) per launch of the attention kernel on this workload, from the
 # ncu capture summarised in profiles/attn_fwd_sm100_ulysses_s44160.md; valid only for the
 # kernel version named there (set to None whenever the kernel changes until re-captured).
-ATTN_TRAFFIC_BYTES = 580_206_336 + 172_326_912
+ATTN_TRAFFIC_BYTES = None
 L2_NOTE = ("inputs larger than L2: each step streams 543 MB of Q/K/V shards plus 724 MB of "
            "permute traffic through the 126 MB L2")
 

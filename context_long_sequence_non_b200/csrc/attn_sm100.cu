@@ -50,6 +50,11 @@ constexpr float kLog2e = 1.44269504088896340736f;
 // and the rest through the special-function unit (ex2), which would otherwise be
 // co-critical with the tensor core (one ex2 per score, 16 per clock per SM).
 constexpr int kPolyPairs = 2;
+// P handoff granularity: each block's P is stored and handed to the issuer in this many
+// key chunks, so that O += P V of the first chunks runs while the rest of P is computed.
+constexpr int kPChunks = 2;
+constexpr int kChunkPairs = kBlockN / 2 / kPChunks;  // bf16 pairs (TMEM columns) per chunk
+static_assert(kChunkPairs == 16 || kChunkPairs == 32, "P chunks of 32 or 64 keys");
 
 template <int D>
 struct Geometry {
@@ -70,7 +75,7 @@ struct __align__(8) Barriers {
   uint64_t full[kSlots];
   uint64_t empty[kSlots];
   uint64_t s_full[2];
-  uint64_t p_full[2];
+  uint64_t p_part[2][kPChunks];  // P chunk c of Q tile t stored (chunk 0: O rescaled too)
   uint64_t o_full;
   uint64_t drain;
 };
@@ -138,7 +143,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(smem_u32(&bars.s_full[t]), 1);
-      mbar_init(smem_u32(&bars.p_full[t]), kBlockM);
+      for (int c = 0; c < kPChunks; ++c)
+        mbar_init(smem_u32(&bars.p_part[t][c]), 4);  // one arrive per softmax warp
     }
     mbar_init(smem_u32(&bars.o_full), 1);
     mbar_init(smem_u32(&bars.drain), 1);
@@ -174,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_s = tmem + lane_bits + uint32_t(tile * kBlockN);
     const uint32_t t_o = tmem + lane_bits + uint32_t(2 * kBlockN + tile * D);
     const uint32_t bar_s = smem_u32(&bars.s_full[tile]);
-    const uint32_t bar_p = smem_u32(&bars.p_full[tile]);
+    const uint32_t bar_p0 = smem_u32(&bars.p_part[tile][0]);  // chunk c at + 8 c
     float m = -INFINITY;  // running (possibly stale) max of x = s * scale * log2(e)
     float l = 0.f;        // running sum of 2^(x - m)
     bool ok = true;
@@ -234,16 +240,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // p = 2^(x * scale_log2 - m): most pairs on the special-function unit, kPolyPairs of
       // every 8 pairs on the FMA pipe (exp2_poly2); p rounded to bf16 for the PV product and
-      // written over S as bf16 pairs; the row sum keeps the unrounded fp32 p
+      // written over S as bf16 pairs; the row sum keeps the unrounded fp32 p.  The keys go
+      // in kPChunks chunks with one handoff each, so that the issuer runs O += P V of the
+      // first chunks while the rest of P is computed.
       const float2 sl2 = make_float2(scale_log2, scale_log2);
       const float2 nm2 = make_float2(-m, -m);
       float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
+      for (int part = 0; part < kPChunks; ++part) {
+        uint32_t pk[kChunkPairs];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c = half * 64 + 2 * e;
+        for (int e = 0; e < kChunkPairs; ++e) {
+          const int c = 2 * (part * kChunkPairs + e);
           const float2 t = ffma2(make_float2(x[c], x[c + 1]), sl2, nm2);
           float2 pv;
           if ((e & 7) >= 8 - kPolyPairs) {
@@ -256,30 +264,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           else acc0 = fadd2(acc0, pv);
           pk[e] = pack_bf16x2(pv.x, pv.y);
         }
-        tmem_st32(t_s + half * 32, pk);
+        tmem_st_any(t_s + part * kChunkPairs, pk);
+        if (part == 0 && rescale) {
+          // rescale this warp's O rows by alpha before the first PV chunk accumulates into
+          // them: PV of the previous block has completed (the issuer committed this
+          // block's S after it), and no PV of this block starts before the arrive below
+          const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+          for (int oc = 0; oc < D / 32; ++oc) {
+            uint32_t r[32];
+            tmem_ld32(t_o + oc * 32, r);
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+              const float2 o =
+                  fmul2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), a2);
+              r[c] = __float_as_uint(o.x);
+              r[c + 1] = __float_as_uint(o.y);
+            }
+            tmem_st32(t_o + oc * 32, r);
+          }
+        }
+        // hand this chunk over: every lane's TMEM stores complete, then one arrive per warp
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_p0 + 8 * part);
       }
       const float2 acc = fadd2(acc0, acc1);
       l += acc.x + acc.y;
-      if (rescale) {
-        // rescale this warp's O rows by alpha: PV of the previous block has completed
-        // (the issuer committed this block's S after it) and the next PV waits for
-        // p_full, so nothing else touches O now
-        uint32_t r[D];
-        if constexpr (D == 128) tmem_ld128(t_o, r);
-        else tmem_ld64(t_o, r);
-        const float2 a2 = make_float2(alpha, alpha);
-#pragma unroll
-        for (int c = 0; c < D; c += 2) {
-          const float2 o = fmul2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), a2);
-          r[c] = __float_as_uint(o.x);
-          r[c + 1] = __float_as_uint(o.y);
-        }
-        if constexpr (D == 128) tmem_st128(t_o, r);
-        else tmem_st64(t_o, r);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar_p);
     }
 
     // ------------------------------------------------------------------ epilogue
@@ -444,15 +456,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // O_t += P_t V over the 128 keys in K=16 steps; P from TMEM (8 columns = 16 bf16
       // per step), V MN-major: 16 key rows = 2 KB per step, the d halves one box apart
-      auto issue_pv = [&](int t, uint32_t v_addr, bool accumulate) {
+      constexpr int kStepsPerChunk = kBlockN / 16 / kPChunks;
+      auto issue_pv_chunk = [&](int t, uint32_t v_addr, bool accumulate, int part) {
 #pragma unroll
-        for (int kk = 0; kk < kBlockN / 16; ++kk) {
+        for (int kk = part * kStepsPerChunk; kk < (part + 1) * kStepsPerChunk; ++kk) {
           mma_ts(t_o[t], t_s[t] + kk * 8, sdesc_sw128(v_addr + kk * 16 * 128, G::kBoxBytes, 1024),
                  idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
         }
       };
       auto slot_addr = [&](int use) {
         return smem_base + G::kOffSlots + (use % kSlots) * G::kTileBytes;
+      };
+      // O_t += P_t V, chunk by chunk as the softmax warps hand P over
+      auto issue_pv = [&](int t, uint32_t v_addr, int j) {
+#pragma unroll
+        for (int part = 0; part < kPChunks; ++part) {
+          if (!mbar_wait(smem_u32(&bars.p_part[t][part]), uint32_t(j) & 1u, abort_flag, err,
+                         wait_limit))
+            return false;
+          tc_fence_after();
+          issue_pv_chunk(t, v_addr, j > 0 || part > 0, part);
+        }
+        return true;
       };
       auto wait_full = [&](int use) {
         return mbar_wait(smem_u32(&bars.full[use % kSlots]), uint32_t(use / kSlots) & 1u,
@@ -472,18 +497,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int use_v = 2 * j + 1, use_k = 2 * j + 2;
         const bool more = j + 1 < n_kv;
         if (!(ok = wait_full(use_v))) break;
-        if (!(ok = mbar_wait(smem_u32(&bars.p_full[0]), j & 1, abort_flag, err, wait_limit))) break;
-        tc_fence_after();
-        issue_pv(0, slot_addr(use_v), j > 0);
+        if (!(ok = issue_pv(0, slot_addr(use_v), j))) break;
         if (more) {
           if (!(ok = wait_full(use_k))) break;
           tc_fence_after();
           issue_qk(0, slot_addr(use_k));
           tc_commit(smem_u32(&bars.s_full[0]));
         }
-        if (!(ok = mbar_wait(smem_u32(&bars.p_full[1]), j & 1, abort_flag, err, wait_limit))) break;
-        tc_fence_after();
-        issue_pv(1, slot_addr(use_v), j > 0);
+        if (!(ok = issue_pv(1, slot_addr(use_v), j))) break;
         tc_commit(smem_u32(&bars.empty[use_v % kSlots]));
         if (more) {
           issue_qk(1, slot_addr(use_k));

@@ -226,6 +226,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 
 // Registers -> 32 consecutive TMEM columns of this thread's lane (completion awaited by
 // tmem_st_wait()).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -367,6 +377,14 @@ __device__ __forceinline__ void tmem_st128(uint32_t taddr, const uint32_t (&r)[1
         "r"(r[117]), "r"(r[118]), "r"(r[119]), "r"(r[120]), "r"(r[121]), "r"(r[122]),
         "r"(r[123]), "r"(r[124]), "r"(r[125]), "r"(r[126]), "r"(r[127])
       : "memory");
+}
+
+// the store of the width an array has (16 or 32 columns)
+__device__ __forceinline__ void tmem_st_any(uint32_t taddr, const uint32_t (&r)[16]) {
+  tmem_st16(taddr, r);
+}
+__device__ __forceinline__ void tmem_st_any(uint32_t taddr, const uint32_t (&r)[32]) {
+  tmem_st32(taddr, r);
 }
 
 // Warpgroup register re-partitioning (all four warps of a warpgroup execute it).  The
