@@ -7,7 +7,9 @@ of what the per-rank context-parallel attention path computes:
 * the exact merge of two partial (O, LSE) results over disjoint key sets, which is
   the Ring Attention step (``ref.merge``),
 * the DeepSpeed-Ulysses sequence<->head re-partition run over P virtual ranks
-  (``ref.seq2head`` / ``ref.head2seq``).
+  (``ref.seq2head`` / ``ref.head2seq``),
+* the attention_mdtrt sample's RMSNorm of the Q and K head rows, in the float32 the
+  page fixes (``ref.rmsnorm_heads``).
 
 Sources (the pages print prose and figures only, no formula; each function states
 the reading it takes):

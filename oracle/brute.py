@@ -66,3 +66,15 @@ def head2seq(src, p):
                     for e in range(d):
                         dst[r][s][g * hp + j][e] = src[g][r * s_l + s][j][e]
     return dst
+
+
+def rmsnorm_heads(x, gamma, eps=1e-6, out_scale=1.0):
+    """The attention_mdtrt sample's Q/K RMSNorm (模型的核心结构) by explicit loops in
+    float64: y[..][d] = x[..][d] / sqrt(fsum(x^2) / D + eps) * gamma[d] * out_scale.
+    ``x`` is a nested list whose innermost lists are head rows of length D."""
+    if hasattr(x[0], "__len__"):  # not yet at a head row: recurse
+        return [rmsnorm_heads(sub, gamma, eps, out_scale) for sub in x]
+    row = [float(t) for t in x]
+    dn = len(row)
+    rms = math.sqrt(math.fsum(t * t for t in row) / dn + eps)
+    return [row[d] / rms * float(gamma[d]) * out_scale for d in range(dn)]

@@ -224,3 +224,31 @@ def ulysses_attention(q_shards, k_shards, v_shards, p: int, scale: float):
     o, lse = attention(qh, kh, vh, scale)
     return head2seq(o, p), lse
 
+
+
+def rmsnorm_heads(x, gamma, eps: float = 1e-6, out_scale: float = 1.0) -> np.ndarray:
+    """RMSNorm of every head row of Q or K, as the attention_mdtrt sample applies it.
+
+    "TensorRT 多设备注意力推理实战" (guide to the attention_mdtrt sample), section
+    模型的核心结构: after Q and K are reshaped to heads (seq, batch, 32, 128), each is
+    normalised in fp32 as x * rsqrt(mean(x^2) + eps) with eps = 1e-6, multiplied by a
+    weight, and cast back to a 16-bit type; Q and K are then each scaled by
+    sqrt(sqrt(1/HEAD_DIM)) before QK^T.
+
+    Readings: the mean runs over the last axis (the head dimension D); one weight vector
+    ``gamma[D]`` serves every head and token; the arithmetic is float32 because the page
+    fixes it (x*r first, then *gamma, then *out_scale, each rounded to float32);
+    ``out_scale`` is the optional split scale applied before the cast (1 when the scale
+    is applied to the logits instead, as 1/sqrt(D)).  Returns float32 values *before*
+    the cast to 16 bits; the caller rounds (bf16 round-to-nearest-even here, where the
+    sample uses fp16).  ``x`` is ``[..., D]``.
+    """
+    x32 = np.asarray(_f64(x), dtype=np.float32)  # exact for bf16/fp32 inputs
+    g32 = np.asarray(_f64(gamma), dtype=np.float32)
+    assert g32.shape == (x32.shape[-1],)
+    ms = np.mean(np.square(x32), axis=-1, dtype=np.float32, keepdims=True)
+    r = np.float32(1.0) / np.sqrt(ms + np.float32(eps))
+    y = (x32 * r) * g32
+    if out_scale != 1.0:
+        y = y * np.float32(out_scale)
+    return y.astype(np.float32)
