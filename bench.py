@@ -40,13 +40,23 @@ WORKLOAD = W.WORKLOADS[4]
 # DRAM bytes (read + write) per launch of the attention kernel on this workload, from the
 # ncu capture summarised in profiles/attn_fwd_sm100_ulysses_s44160.md; valid only for the
 # kernel version named there (set to None whenever the kernel changes until re-captured).
-ATTN_TRAFFIC_BYTES = None
+ATTN_TRAFFIC_BYTES = 597_763_840 + 168_522_496
 L2_NOTE = ("inputs larger than L2: each step streams 543 MB of Q/K/V shards plus 724 MB of "
            "permute traffic through the 126 MB L2")
 
 
-def workload_config():
+def workload_config(qk_norm=False):
     w = WORKLOAD
+    if qk_norm:
+        return {
+            "workload": ("ulysses-cp8-s44160 with Q/K RMSNorm: P=8 virtual ranks x [5520 tokens]"
+                         "[16 heads][128] bf16 Q/K/V, one seq2head launch for Q/K/V with the "
+                         "RMSNorm of every Q and K head row fused in (eps 1e-6, float32 weights) + "
+                         "non-causal attention + head2seq"),
+            "B": w.B, "H": w.H, "S": w.Sq, "D": w.D, "P": w.P,
+            "inputs": "iid N(0,1), torch.Generator seed 4000, rounded to bf16; weights 1+0.1 N(0,1)",
+            "l2": L2_NOTE,
+        }
     return {
         "workload": (f"ulysses-cp8-s44160: P=8 virtual ranks x [5520 tokens][16 heads][128] bf16 "
                      f"Q/K/V, 3x seq2head + non-causal attention (8 head groups x 2 heads, "
@@ -184,12 +194,18 @@ def run_ours(args, world, rank, local):
     plan = UlyssesPlan(P, S_l, H, w.D, device=dev)
     stream = torch.cuda.current_stream(dev)
     flops = w.attn_flops
-    launches_per_step = 5
+    launches_per_step = 3 if args.qk_norm else 5
+    if args.qk_norm:  # the sample's Q/K RMSNorm fused into one Q/K/V seq2head launch
+        gq = W.norm_weights(w.D, seed=41).to(dev)
+        gk = W.norm_weights(w.D, seed=42).to(dev)
 
     def step(ev_attn=None):
-        cp.seq2head(q, P, out=plan.qh)
-        cp.seq2head(k, P, out=plan.kh)
-        cp.seq2head(v, P, out=plan.vh)
+        if args.qk_norm:
+            cp.seq2head_qkv_norm(q, k, v, P, gq, gk, out=(plan.qh, plan.kh, plan.vh))
+        else:
+            cp.seq2head(q, P, out=plan.qh)
+            cp.seq2head(k, P, out=plan.kh)
+            cp.seq2head(v, P, out=plan.vh)
         if ev_attn is not None:
             ev_attn[0].record(stream)
         cp.fwd(plan.qh, plan.kh, plan.vh, out=plan.oh, lse=plan.lse, scale=w.softmax_scale)
@@ -249,7 +265,7 @@ def run_ours(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(max_ms / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(),
+        "config": workload_config(args.qk_norm),
         "frac_of_dense_bf16_peak": round(value / peak, 4),
         "roofline": {
             "bound": "tensor", "kernel": "attn_fwd_sm100_kernel<128,false>",
@@ -377,6 +393,21 @@ def next_paths(cp, w, q, k, v, plan, dev, stream):
     res["seq2head_qkv"] = {"ms": round(ms, 4), "bytes": nbytes,
                            "GB/s": round(nbytes / ms / 1e6, 1),
                            "frac_of_hbm": round(nbytes / ms / 1e6 / peaks["hbm_gbs"], 4)}
+    # the sample's Q/K RMSNorm fused into that launch (same bytes), and standalone in place
+    gq = W.norm_weights(w.D, seed=41).to(dev)
+    gk = W.norm_weights(w.D, seed=42).to(dev)
+    ms = timed(lambda: cp.seq2head_qkv_norm(q, k, v, w.P, gq, gk, out=(plan.qh, plan.kh, plan.vh)))
+    res["seq2head_qkv_norm"] = {"ms": round(ms, 4), "bytes": nbytes,
+                                "GB/s": round(nbytes / ms / 1e6, 1),
+                                "frac_of_hbm": round(nbytes / ms / 1e6 / peaks["hbm_gbs"], 4),
+                                "what": "seq2head of Q, K, V with RMSNorm of Q and K head rows"}
+    qn = q.clone()
+    nb1 = 2 * qn.numel() * qn.element_size()
+    ms = timed(lambda: cp.rmsnorm(qn, gq, out=qn))
+    res["rmsnorm"] = {"ms": round(ms, 4), "bytes": nb1, "GB/s": round(nb1 / ms / 1e6, 1),
+                      "frac_of_hbm": round(nb1 / ms / 1e6 / peaks["hbm_gbs"], 4),
+                      "what": "RMSNorm of [8][5520][16][128] bf16 head rows, in place"}
+    del qn
     w3 = W.WORKLOADS[3]
     x3 = W.make_inputs(w3)
     q3, k3, v3 = (x3[n].to(dev) for n in ("q", "k", "v"))
@@ -541,6 +572,9 @@ def main(argv=None):
     ap.add_argument("--profile", action="store_true",
                     help="for profiler captures: run only warm-up + timed steps (no aux "
                          "kernels, no end-to-end pass, no CPU baseline)")
+    ap.add_argument("--qk-norm", action="store_true",
+                    help="step variant: Q/K RMSNorm fused into one Q/K/V seq2head launch "
+                         "(not the headline step; for profiling that kernel)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")

@@ -25,10 +25,12 @@ from ._binding import (  # noqa: F401
     lib,
     library_path,
     merge,
+    rmsnorm,
     selftest_exp2,
     selftest_wait_timeout,
     seq2head,
     seq2head_qkv,
+    seq2head_qkv_norm,
     status_str,
     version,
 )

@@ -58,6 +58,9 @@ def lib() -> ctypes.CDLL:
             L.cpattn_seq2head.argtypes = [vp, vp, i, i, i, i, i, vp]
             L.cpattn_head2seq.argtypes = [vp, vp, i, i, i, i, i, vp]
             L.cpattn_seq2head_qkv.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
+            L.cpattn_rmsnorm.argtypes = [vp, vp, vp, i, i, f, f, vp]
+            L.cpattn_seq2head_qkv_norm.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f,
+                                                   f, vp]
             L.cpattn_status_str.argtypes = [i]
             L.cpattn_status_str.restype = ctypes.c_char_p
             L.cpattn_device_error.argtypes = []
@@ -250,6 +253,45 @@ def seq2head_qkv(q, k, v, P, out=None, stream=None):
     st = lib().cpattn_seq2head_qkv(_ptr(q), _ptr(k), _ptr(v), *(_ptr(t) for t in out), P, S_l, H,
                                    D, q.element_size(), _stream(stream))
     _check(st, "cpattn_seq2head_qkv")
+    return out
+
+
+def rmsnorm(x, gamma, eps=1e-6, out_scale=1.0, out=None, stream=None):
+    """RMSNorm of every head row (last axis, D) of a bf16 tensor with fp32 weights
+    ``gamma[D]``; ``out=x`` normalises in place.  See cpattn_rmsnorm."""
+    if x.dtype != torch.bfloat16 or gamma.dtype != torch.float32 or gamma.shape != (x.shape[-1],):
+        raise ValueError("x must be bf16 [..., D] and gamma float32 [D]")
+    if out is None:
+        out = torch.empty_like(x)
+    if out.shape != x.shape or out.dtype != x.dtype:
+        raise ValueError("out must match x")
+    _need_cuda(x, gamma, out)
+    D = x.shape[-1]
+    st = lib().cpattn_rmsnorm(_ptr(x), _ptr(out), _ptr(gamma), x.numel() // D, D, float(eps),
+                              float(out_scale), _stream(stream))
+    _check(st, "cpattn_rmsnorm")
+    return out
+
+
+def seq2head_qkv_norm(q, k, v, P, gamma_q, gamma_k, eps=1e-6, out_scale=1.0, out=None,
+                      stream=None):
+    """seq2head of Q, K, V in one launch with Q and K head rows RMS-normalised on the way
+    (weights gamma_q / gamma_k, float32 [D]); ``out`` is an optional (qh, kh, vh) triple."""
+    P_, S_l, H, D = q.shape
+    if P_ != P or k.shape != q.shape or v.shape != q.shape or any(
+            t.dtype != torch.bfloat16 for t in (q, k, v)):
+        raise ValueError("q, k, v must be same-shaped bf16 [P][S_l][H][D] tensors")
+    for g in (gamma_q, gamma_k):
+        if g.dtype != torch.float32 or g.shape != (D,):
+            raise ValueError("gamma_q and gamma_k must be float32 [D]")
+    if out is None:
+        out = tuple(torch.empty((P, P * S_l, H // P, D), dtype=q.dtype, device=q.device)
+                    for _ in range(3))
+    _need_cuda(q, k, v, gamma_q, gamma_k, *out)
+    st = lib().cpattn_seq2head_qkv_norm(_ptr(q), _ptr(k), _ptr(v), *(_ptr(t) for t in out),
+                                        _ptr(gamma_q), _ptr(gamma_k), P, S_l, H, D, float(eps),
+                                        float(out_scale), _stream(stream))
+    _check(st, "cpattn_seq2head_qkv_norm")
     return out
 
 

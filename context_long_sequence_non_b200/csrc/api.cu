@@ -346,6 +346,58 @@ int cpattn_seq2head_qkv(const void* q, const void* k, const void* v, void* qh, v
                                                reinterpret_cast<cudaStream_t>(stream)));
 }
 
+static bool norm_dim_ok(int D) { return D >= 8 && D <= 256 && (D & (D - 1)) == 0; }
+
+static int norm_scalars_ok(float eps, float out_scale) {
+  if (!(eps >= 0.0f) || !std::isfinite(eps) || !std::isfinite(out_scale)) return CPATTN_ERR_SHAPE;
+  return CPATTN_OK;
+}
+
+int cpattn_rmsnorm(const void* x, void* y, const float* gamma, int rows, int D, float eps,
+                   float out_scale, cpattn_stream_t stream) {
+  if (rows < 0 || !norm_dim_ok(D)) return CPATTN_ERR_SHAPE;
+  const int sc = norm_scalars_ok(eps, out_scale);
+  if (sc != CPATTN_OK) return sc;
+  if (rows == 0) return CPATTN_OK;  // nothing is read or written: pointers are not checked
+  if ((long long)rows * (D / 8) > 0x7fffffffLL - 256) return CPATTN_ERR_SHAPE;  // 32-bit vectors
+  if (x == nullptr || y == nullptr || gamma == nullptr) return CPATTN_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(gamma, 16)) return CPATTN_ERR_ALIGN;
+  const size_t bytes = size_t(rows) * D * 2;
+  if (x != y && overlap(x, bytes, y, bytes)) return CPATTN_ERR_SHAPE;  // in place or disjoint
+  if (overlap(gamma, size_t(D) * 4, y, bytes)) return CPATTN_ERR_SHAPE;
+  return cuda_status(cpattn::launch_rmsnorm(x, y, gamma, rows, D, eps, out_scale,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int cpattn_seq2head_qkv_norm(const void* q, const void* k, const void* v, void* qh, void* kh,
+                             void* vh, const float* gamma_q, const float* gamma_k, int P,
+                             int S_local, int H, int D, float eps, float out_scale,
+                             cpattn_stream_t stream) {
+  if (!norm_dim_ok(D)) return CPATTN_ERR_SHAPE;
+  const int sc = norm_scalars_ok(eps, out_scale);
+  if (sc != CPATTN_OK) return sc;
+  const void* src[3] = {q, k, v};
+  void* dst[3] = {qh, kh, vh};
+  long long run_vec = 0;
+  for (int t = 0; t < 3; ++t) {
+    const int st = permute_args(src[t], dst[t], P, S_local, H, D, 2, &run_vec);
+    if (st != CPATTN_OK) return st;
+  }
+  if (gamma_q == nullptr || gamma_k == nullptr) return CPATTN_ERR_NULL;
+  if (!aligned(gamma_q, 16) || !aligned(gamma_k, 16)) return CPATTN_ERR_ALIGN;
+  const size_t bytes = size_t(P) * S_local * H * D * 2;
+  for (int a = 0; a < 3; ++a) {
+    for (int c = 0; c < 3; ++c)
+      if ((a != c && overlap(dst[a], bytes, dst[c], bytes)) || overlap(dst[a], bytes, src[c], bytes))
+        return CPATTN_ERR_SHAPE;
+    if (overlap(dst[a], bytes, gamma_q, size_t(D) * 4) || overlap(dst[a], bytes, gamma_k, size_t(D) * 4))
+      return CPATTN_ERR_SHAPE;
+  }
+  return cuda_status(cpattn::launch_seq2head_qkv_norm(src, dst, gamma_q, gamma_k, P, S_local, D,
+                                                      run_vec, eps, out_scale,
+                                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int cpattn_head2seq(const void* src, void* dst, int P, int S_local, int H, int D, int elem_bytes,
                     cpattn_stream_t stream) {
   long long run_vec = 0;

@@ -65,6 +65,15 @@ cudaError_t launch_head2seq(const void* src, void* dst, int P, int S_local, long
 // seq2head of n (1..3) same-shaped tensors in one launch.
 cudaError_t launch_seq2head_n(const void* const* src, void* const* dst, int n, int P, int S_local,
                               long long run_vec, cudaStream_t stream);
+// seq2head of Q, K, V in one launch with the RMSNorm of every Q and K head row fused in
+// (src/dst: 3 tensors; D a power of two with D/8 dividing 32).
+cudaError_t launch_seq2head_qkv_norm(const void* const* src, void* const* dst, const float* gamma_q,
+                                     const float* gamma_k, int P, int S_local, int D,
+                                     long long run_vec, float eps, float out_scale,
+                                     cudaStream_t stream);
+// RMSNorm of `rows` head rows of D bf16 (x and y may be the same buffer).
+cudaError_t launch_rmsnorm(const void* x, void* y, const float* gamma, long long rows, int D,
+                           float eps, float out_scale, cudaStream_t stream);
 
 // One CTA waiting on an mbarrier nothing completes, with the attention kernel's bounded wait.
 cudaError_t launch_wait_timeout_selftest(int* err, long long limit, cudaStream_t stream);

@@ -277,8 +277,68 @@ struct PermuteSet {
   uint4* dst[3];
 };
 
-template <bool kToHead>
-__global__ void __launch_bounds__(kPermThreads) permute_kernel(const __grid_constant__ PermuteSet set,
+// Optional RMSNorm of every head row on the way through (the Q/K norm of the
+// attention_mdtrt sample, section 模型的核心结构): y = bf16(((x * r) * gamma[d]) * out_scale)
+// with r = 1 / sqrt(mean(x^2) + eps), all in fp32.  A head row of D bf16 is row_vec = D/8
+// vectors held by row_vec consecutive lanes (32 % row_vec == 0, and runs and 32-vector
+// chunks start on head-row boundaries), so its sum of squares is a shuffle reduction and
+// the head-dim slice a lane sees, (lane % row_vec) * 8 .. + 7, is the same for every item:
+// its 8 weights are loaded once.
+struct RowNorm {
+  const float* gamma[3];  // per tensor of the set; nullptr = copied unchanged
+  int row_vec;
+  float inv_d, eps, out_scale;
+};
+
+// 1/sqrt(a) for a > 0: the special-function unit's estimate refined by one Newton step on
+// f(y) = 1/y^2 - a (y' = y * (3 - a y^2) / 2), which brings it to about an ulp of the
+// float32 1/sqrt(a) for every positive finite a (subnormal a included).
+__device__ __forceinline__ float rsqrt_refined(float a) {
+  float y;
+  asm("rsqrt.approx.f32 %0, %1;" : "=f"(y) : "f"(a));
+  const float hy = 0.5f * y;
+  return fmaf(hy, fmaf(-a * y, y, 1.0f), y);  // y + (y/2)(1 - a y^2)
+}
+
+__device__ __forceinline__ void load_gamma8(const float* __restrict__ gamma, int d0, float (&g)[8]) {
+  const float4 g0 = __ldg(reinterpret_cast<const float4*>(gamma + d0));
+  const float4 g1 = __ldg(reinterpret_cast<const float4*>(gamma + d0 + 4));
+  g[0] = g0.x; g[1] = g0.y; g[2] = g0.z; g[3] = g0.w;
+  g[4] = g1.x; g[5] = g1.y; g[6] = g1.z; g[7] = g1.w;
+}
+
+// Normalise the 8 elements of one 16-byte vector; every lane of the warp must call it
+// (dead lanes with live = false contribute nothing and get `in` back).
+__device__ __forceinline__ uint4 rms_normalise(uint4 in, bool live, int row_vec, float inv_d,
+                                               float eps, float out_scale, const float (&g)[8]) {
+  const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+  float f[8];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    f[2 * t] = live ? __uint_as_float(w[t] << 16) : 0.f;  // bf16 -> fp32 is exact
+    f[2 * t + 1] = live ? __uint_as_float(w[t] & 0xFFFF0000u) : 0.f;
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+  for (int o = 1; o < row_vec; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float a = ss * inv_d + eps;
+  const float r = a > 0.f ? rsqrt_refined(a) : 0.f;  // an all-zero row with eps = 0 stays 0
+  if (!live) return in;
+  float y[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) y[e] = (f[e] * r) * g[e];
+  if (out_scale != 1.0f) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[e] *= out_scale;
+  }
+  return make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                    pack_bf16x2(y[6], y[7]));
+}
+
+template <bool kToHead, bool kNorm>
+__global__ void __launch_bounds__(kPermThreads, kNorm ? 5 : 1) permute_kernel(const __grid_constant__ PermuteSet set,
+                                                                const __grid_constant__ RowNorm nrm,
                                                                 int P, int S_l, int run_vec,
                                                                 int chunks, int n_items) {
   // blockIdx.y picks the tensor (uniform per block); item = (dst row, 32-vector chunk)
@@ -287,32 +347,57 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const __grid_cons
   const int lane = threadIdx.x & 31;
   const int warp = int((blockIdx.x * kPermThreads + threadIdx.x) >> 5);
   const int n_warps = int((gridDim.x * kPermThreads) >> 5);
+  const float* __restrict__ gamma = kNorm ? nrm.gamma[blockIdx.y] : nullptr;  // per block
+  float g[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (kNorm && gamma != nullptr) load_gamma8(gamma, (lane % nrm.row_vec) * 8, g);
   for (int it0 = warp * kPermUnroll; it0 < n_items; it0 += n_warps * kPermUnroll) {
     uint4 buf[kPermUnroll];
     long long dst_off[kPermUnroll];
     bool live[kPermUnroll];
+    // The warp's items it0 .. it0+kPermUnroll-1 are consecutive: divide once for the
+    // first, then step the mixed-radix digits of the dst row.  seq2head: n = A(g, r, s),
+    // digits (d0, d1, d2) = (s, r, g); head2seq: n = Bq(g, r, s), digits (g, s, r).
+    int n = it0 / chunks;  // dst row
+    int c = it0 - n * chunks;
+    int d0, d1, d2;
+    if (kToHead) {
+      const int q = n / S_l;
+      d0 = n - q * S_l;
+      d2 = q / P;
+      d1 = q - d2 * P;
+    } else {
+      const int q = n / P;
+      d0 = n - q * P;
+      d2 = q / S_l;
+      d1 = q - d2 * S_l;
+    }
+    const int R0 = kToHead ? S_l : P, R1 = kToHead ? P : S_l;
 #pragma unroll
     for (int u = 0; u < kPermUnroll; ++u) {
-      const int it = it0 + u;
-      const int n = it / chunks;  // dst row
-      const int v = (it - n * chunks) * 32 + lane;
-      live[u] = it < n_items && v < run_vec;
-      int src_row;
-      if (kToHead) {  // n = A(g, r, s)
-        const int gr = n / S_l;
-        const int s = n - gr * S_l;
-        const int g = gr / P;
-        const int r = gr - g * P;
-        src_row = (r * S_l + s) * P + g;
-      } else {  // n = Bq(g, r, s)
-        const int rs = n / P;
-        const int g = n - rs * P;
-        const int r = rs / S_l;
-        const int s = rs - r * S_l;
-        src_row = (g * P + r) * S_l + s;
-      }
+      const int v = c * 32 + lane;
+      live[u] = it0 + u < n_items && v < run_vec;
+      const int src_row = kToHead ? (d1 * S_l + d0) * P + d2   // Bq(g, r, s)
+                                  : (d0 * P + d2) * S_l + d1;  // A(g, r, s)
       dst_off[u] = (long long)n * run_vec + v;
       if (live[u]) buf[u] = src[(long long)src_row * run_vec + v];
+      if (++c == chunks) {  // next item: next chunk, else the next dst row
+        c = 0;
+        ++n;
+        if (++d0 == R0) {
+          d0 = 0;
+          if (++d1 == R1) {
+            d1 = 0;
+            ++d2;
+          }
+        }
+      }
+    }
+    if constexpr (kNorm) {
+      if (gamma != nullptr) {
+#pragma unroll
+        for (int u = 0; u < kPermUnroll; ++u)
+          buf[u] = rms_normalise(buf[u], live[u], nrm.row_vec, nrm.inv_d, nrm.eps, nrm.out_scale, g);
+      }
     }
 #pragma unroll
     for (int u = 0; u < kPermUnroll; ++u)
@@ -460,7 +545,7 @@ cudaError_t launch_combine(const void* part_o, const float* part_lse, int n, voi
 
 static cudaError_t launch_permute(bool to_head, const void* const* src, void* const* dst,
                                   int n_tensors, int P, int S_local, long long run_vec,
-                                  cudaStream_t stream) {
+                                  cudaStream_t stream, const RowNorm* nrm = nullptr) {
   PermuteSet set{};
   for (int t = 0; t < 3; ++t) {
     const int u = t < n_tensors ? t : 0;
@@ -476,12 +561,85 @@ static cudaError_t launch_permute(bool to_head, const void* const* src, void* co
   const long long cap = (long long)sm_count() * 8 / n_tensors + 1;
   const long long blocks = blocks_needed < cap ? blocks_needed : cap;
   const dim3 grid{unsigned(blocks), unsigned(n_tensors), 1u};
-  if (to_head)
-    permute_kernel<true><<<grid, kPermThreads, 0, stream>>>(set, P, S_local, int(run_vec), chunks,
-                                                            int(n_items));
+  const RowNorm none{};
+  if (nrm != nullptr)
+    permute_kernel<true, true><<<grid, kPermThreads, 0, stream>>>(set, *nrm, P, S_local,
+                                                                  int(run_vec), chunks, int(n_items));
+  else if (to_head)
+    permute_kernel<true, false><<<grid, kPermThreads, 0, stream>>>(set, none, P, S_local,
+                                                                   int(run_vec), chunks, int(n_items));
   else
-    permute_kernel<false><<<grid, kPermThreads, 0, stream>>>(set, P, S_local, int(run_vec), chunks,
-                                                             int(n_items));
+    permute_kernel<false, false><<<grid, kPermThreads, 0, stream>>>(set, none, P, S_local,
+                                                                    int(run_vec), chunks, int(n_items));
+  return cudaGetLastError();
+}
+
+static RowNorm row_norm(const float* g0, const float* g1, const float* g2, int D, float eps,
+                        float out_scale) {
+  RowNorm n{};
+  n.gamma[0] = g0;
+  n.gamma[1] = g1;
+  n.gamma[2] = g2;
+  n.row_vec = D / 8;
+  n.inv_d = 1.0f / float(D);  // D is a power of two: x * inv_d == x / D exactly
+  n.eps = eps;
+  n.out_scale = out_scale;
+  return n;
+}
+
+cudaError_t launch_seq2head_qkv_norm(const void* const* src, void* const* dst, const float* gamma_q,
+                                     const float* gamma_k, int P, int S_local, int D,
+                                     long long run_vec, float eps, float out_scale,
+                                     cudaStream_t stream) {
+  const RowNorm n = row_norm(gamma_q, gamma_k, nullptr, D, eps, out_scale);
+  return launch_permute(true, src, dst, 3, P, S_local, run_vec, stream, &n);
+}
+
+// Standalone RMSNorm over a flat [rows][D] array: item = 32 consecutive vectors (32/row_vec
+// whole head rows), kPermUnroll items per warp in flight; same arithmetic as the fused form.
+__global__ void __launch_bounds__(kPermThreads, 5) rmsnorm_kernel(const uint4* __restrict__ x,
+                                                                  uint4* __restrict__ y,
+                                                                  const float* __restrict__ gamma,
+                                                                  int n_vec, int row_vec,
+                                                                  float inv_d, float eps,
+                                                                  float out_scale) {
+  const int lane = threadIdx.x & 31;
+  const int warp = int((blockIdx.x * kPermThreads + threadIdx.x) >> 5);
+  const int n_warps = int((gridDim.x * kPermThreads) >> 5);
+  float g[8];
+  load_gamma8(gamma, (lane % row_vec) * 8, g);
+  const int n_items = (n_vec + 31) >> 5;
+  for (int it0 = warp * kPermUnroll; it0 < n_items; it0 += n_warps * kPermUnroll) {
+    uint4 buf[kPermUnroll];
+    bool live[kPermUnroll];
+#pragma unroll
+    for (int u = 0; u < kPermUnroll; ++u) {
+      const int v = ((it0 + u) << 5) + lane;  // < 2^31: n_vec + 31 + 32 * kPermUnroll fits
+      live[u] = it0 + u < n_items && v < n_vec;
+      if (live[u]) buf[u] = x[v];
+    }
+#pragma unroll
+    for (int u = 0; u < kPermUnroll; ++u)
+      buf[u] = rms_normalise(buf[u], live[u], row_vec, inv_d, eps, out_scale, g);
+#pragma unroll
+    for (int u = 0; u < kPermUnroll; ++u)
+      if (live[u]) y[((it0 + u) << 5) + lane] = buf[u];
+  }
+}
+
+cudaError_t launch_rmsnorm(const void* x, void* y, const float* gamma, long long rows, int D,
+                           float eps, float out_scale, cudaStream_t stream) {
+  const int row_vec = D / 8;
+  const long long n_vec = rows * row_vec;
+  // 32-bit vector indices, with room for a warp's last partial item
+  if (n_vec > 0x7fffffffLL - 32 * (kPermUnroll + 1)) return cudaErrorInvalidValue;
+  const long long warps_needed = ((n_vec + 31) / 32 + kPermUnroll - 1) / kPermUnroll;
+  const long long blocks_needed = (warps_needed * 32 + kPermThreads - 1) / kPermThreads;
+  const long long cap = (long long)sm_count() * 8;
+  const long long blocks = blocks_needed < cap ? blocks_needed : cap;
+  rmsnorm_kernel<<<unsigned(blocks), kPermThreads, 0, stream>>>(
+      static_cast<const uint4*>(x), static_cast<uint4*>(y), gamma, int(n_vec), row_vec,
+      1.0f / float(D), eps, out_scale);
   return cudaGetLastError();
 }
 

@@ -71,8 +71,11 @@ class UlyssesPlan:
     Shards are [P][S_l][H][D]; head-grouped buffers [P][P*S_l][H/P][D].
     """
 
-    def __init__(self, P, S_local, H, D, dtype=torch.bfloat16, device="cuda", batched=False):
+    def __init__(self, P, S_local, H, D, dtype=torch.bfloat16, device="cuda", batched=False,
+                 qk_norm=None, norm_eps=1e-6):
         self.batched = batched  # one seq2head launch for Q, K, V together
+        # (gamma_q, gamma_k) float32 [D]: the sample's Q/K RMSNorm fused into that launch
+        self.qk_norm, self.norm_eps = qk_norm, norm_eps
         if H % P:
             raise ValueError("H must be divisible by P")
         self.P, self.S_local, self.H, self.D = P, S_local, H, D
@@ -86,7 +89,10 @@ class UlyssesPlan:
 
     def run(self, q_shards, k_shards, v_shards, scale=None, stream=None):
         P = self.P
-        if self.batched:
+        if self.qk_norm is not None:
+            B.seq2head_qkv_norm(q_shards, k_shards, v_shards, P, *self.qk_norm, eps=self.norm_eps,
+                                out=(self.qh, self.kh, self.vh), stream=stream)
+        elif self.batched:
             B.seq2head_qkv(q_shards, k_shards, v_shards, P, out=(self.qh, self.kh, self.vh),
                            stream=stream)
         else:

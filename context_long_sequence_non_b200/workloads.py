@@ -108,6 +108,14 @@ def make_inputs(w: Workload) -> dict:
     return out
 
 
+def norm_weights(D: int, seed: int) -> torch.Tensor:
+    """float32 [D] RMSNorm weights for the Q/K norm (the sample draws random weights):
+    1 + 0.1 * N(0, 1), seeded."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return 1.0 + 0.1 * torch.randn(D, generator=g, dtype=torch.float32)
+
+
 def random_case(seed: int, B: int, H: int, Sq: int, Skv: int, D: int, dtype: str = "bf16",
                 sigma_qk: float = 1.0, sigma_v: float = 1.0):
     """Generic seeded case for parity tests of ragged and edge shapes."""

@@ -235,6 +235,41 @@ CPATTN_API int cpattn_seq2head_qkv(const void* q, const void* k, const void* v, 
                                    cpattn_stream_t stream);
 
 /*
+ * cpattn_rmsnorm -- the Q/K RMSNorm of the attention_mdtrt sample ("TensorRT 多设备注意力
+ * 推理实战", section 模型的核心结构): after Q and K are split into heads, every head row
+ * is normalised in fp32 as x * rsqrt(mean(x^2) + eps) (eps = 1e-6 there), multiplied by a
+ * weight and cast back to 16 bits.  For each of `rows` head rows of D elements:
+ *   r = 1 / sqrt(sum_d x[d]^2 / D + eps)                  (fp32, IEEE sqrt and division)
+ *   y[d] = bf16_rne(((x[d] * r) * gamma[d]) * out_scale)  (fp32 products)
+ * `out_scale` is the sample's split scale sqrt(sqrt(1/D)) when the caller keeps Q and K
+ * pre-scaled (then pass scale = 1 to cpattn_fwd); pass 1 to apply 1/sqrt(D) to the
+ * logits through cpattn_fwd's `scale` instead (the same product in exact arithmetic).
+ * x, y : [rows][D] bf16 (a [B][S][H][D] tensor is rows = B*S*H); y may be x itself (in
+ * place) but must not overlap it otherwise.  gamma : D float32 weights in device memory,
+ * caller-owned.  D a power of two in [8, 256]; rows >= 0 (rows = 0 is a no-op that reads
+ * no pointer, so empty tensors may pass NULL); eps >= 0 and out_scale finite.  x, y, gamma 16-byte aligned.  The sum of squares is reduced in a
+ * fixed order on the device, so y can differ from a float32 reference that sums in
+ * another order by one bf16 unit in rare ties of the rounding.
+ * Errors: CPATTN_ERR_NULL, _SHAPE, _ALIGN, _CUDA.
+ */
+CPATTN_API int cpattn_rmsnorm(const void* x, void* y, const float* gamma, int rows, int D,
+                              float eps, float out_scale, cpattn_stream_t stream);
+
+/*
+ * cpattn_seq2head_qkv_norm -- cpattn_seq2head_qkv with the RMSNorm of cpattn_rmsnorm
+ * applied to every Q head row (weights gamma_q) and K head row (gamma_k) while they are
+ * copied; V is copied unchanged.  The norm acts on whole head rows and the permute moves
+ * whole head rows, so qh = seq2head(rmsnorm(q)) bit for bit as the two separate calls
+ * give it, at the bytes of the plain permute.  bf16 only (elem_bytes 2); D a power of
+ * two in [8, 256]; other requirements as cpattn_seq2head_qkv and cpattn_rmsnorm.
+ * Errors: CPATTN_ERR_NULL, _SHAPE, _ALIGN, _CUDA.
+ */
+CPATTN_API int cpattn_seq2head_qkv_norm(const void* q, const void* k, const void* v, void* qh,
+                                        void* kh, void* vh, const float* gamma_q,
+                                        const float* gamma_k, int P, int S_local, int H, int D,
+                                        float eps, float out_scale, cpattn_stream_t stream);
+
+/*
  * cpattn_head2seq -- the Ulysses second all-to-all (Fig. 4), exact inverse of
  * cpattn_seq2head:
  *   dst[r][s][g*Hp + j][d] = src[g][r*S_local + s][j][d]

@@ -171,6 +171,42 @@ def test_seq2head_qkv_argument_errors(L):
     assert f(*bad, 2, 4, 16, 128, 2, None) == B.ERR_SHAPE
 
 
+def test_rmsnorm_argument_errors(L):
+    vp = ctypes.c_void_p
+    x, y, g = vp(FAKE), vp(FAKE + 0x1000000), vp(FAKE + 0x2000000)
+    f = L.cpattn_rmsnorm
+    for D in (0, 4, 48, 512, 100):  # powers of two in [8, 256] only
+        assert f(x, y, g, 10, D, 1e-6, 1.0, None) == B.ERR_SHAPE, D
+    assert f(x, y, g, -1, 128, 1e-6, 1.0, None) == B.ERR_SHAPE
+    assert f(x, y, g, 10, 128, -1e-6, 1.0, None) == B.ERR_SHAPE       # eps < 0
+    assert f(x, y, g, 10, 128, float("nan"), 1.0, None) == B.ERR_SHAPE
+    assert f(x, y, g, 10, 128, 1e-6, float("inf"), None) == B.ERR_SHAPE
+    assert f(None, y, g, 10, 128, 1e-6, 1.0, None) == B.ERR_NULL
+    assert f(x, y, None, 10, 128, 1e-6, 1.0, None) == B.ERR_NULL
+    assert f(x, y, vp(FAKE + 0x2000000 + 8), 10, 128, 1e-6, 1.0, None) == B.ERR_ALIGN
+    assert f(x, vp(FAKE + 32), g, 10, 128, 1e-6, 1.0, None) == B.ERR_SHAPE  # partial overlap
+    assert f(x, y, vp(FAKE + 0x1000000 + 64), 10, 128, 1e-6, 1.0, None) == B.ERR_SHAPE  # gamma in y
+    assert f(x, y, g, 0, 128, 1e-6, 1.0, None) == B.OK  # nothing to do, nothing launched
+    assert f(None, None, None, 0, 128, 1e-6, 1.0, None) == B.OK  # empty tensors may be NULL
+    assert f(None, None, None, 0, 96, 1e-6, 1.0, None) == B.ERR_SHAPE  # shape still checked
+
+
+def test_seq2head_qkv_norm_argument_errors(L):
+    vp = ctypes.c_void_p
+    big = 0x1000000
+    ptrs = [vp(FAKE + i * big) for i in range(6)]
+    gq, gk = vp(FAKE + 6 * big), vp(FAKE + 7 * big)
+    f = L.cpattn_seq2head_qkv_norm
+    assert f(*ptrs, gq, gk, 3, 4, 16, 128, 1e-6, 1.0, None) == B.ERR_SHAPE  # H % P
+    assert f(*ptrs, gq, gk, 2, 4, 16, 96, 1e-6, 1.0, None) == B.ERR_SHAPE   # D not a power of 2
+    assert f(*ptrs, gq, gk, 2, 4, 16, 128, -1.0, 1.0, None) == B.ERR_SHAPE  # eps
+    assert f(*ptrs, None, gk, 2, 4, 16, 128, 1e-6, 1.0, None) == B.ERR_NULL
+    assert f(*ptrs, gq, vp(FAKE + 7 * big + 4), 2, 4, 16, 128, 1e-6, 1.0, None) == B.ERR_ALIGN
+    assert f(*ptrs, vp(FAKE + 3 * big + 256), gk, 2, 4, 16, 128, 1e-6, 1.0, None) == B.ERR_SHAPE
+    bad = ptrs[:4] + [vp(FAKE + 5 * big + 32)] + ptrs[5:]
+    assert f(*bad, gq, gk, 2, 4, 16, 128, 1e-6, 1.0, None) == B.ERR_SHAPE
+
+
 def test_selftest_limit_checked(L):
     assert L.cpattn_selftest_wait_timeout(0, None) == B.ERR_SHAPE
     assert L.cpattn_selftest_wait_timeout((1 << 31) + 1, None) == B.ERR_SHAPE
