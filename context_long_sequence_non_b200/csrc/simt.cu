@@ -183,6 +183,62 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
   }
 }
 
+// Rows of at most 32 vectors (bf16 D <= 256, fp32 D <= 128; vpr a power of two): warps
+// stride over items of 32 consecutive vectors = 32/vpr whole rows, kMergeRowsPerThread items
+// in flight, the grid a fixed multiple of the SM count (no tail wave).  A row's lanes all
+// sit in one warp, so an in-place LSE update needs no block barrier: the row's leader lane
+// writes L after, and from, the loads every lane of the warp issued first.
+template <bool kBf16>
+__global__ void __launch_bounds__(kMergeThreads, 4) merge_rows_kernel(
+    const uint4* o_a, const float* lse_a, const uint4* o_b, const float* lse_b, uint4* o,
+    float* lse, int H, int S, int n_vec, int vpr_log2) {
+  const int lane = threadIdx.x & 31;
+  const int warp = int((blockIdx.x * kMergeThreads + threadIdx.x) >> 5);
+  const int n_warps = int((gridDim.x * kMergeThreads) >> 5);
+  const int n_items = (n_vec + 31) >> 5;
+  const bool leader = (lane & ((1 << vpr_log2) - 1)) == 0;
+  for (int it0 = warp * kMergeRowsPerThread; it0 < n_items; it0 += n_warps * kMergeRowsPerThread) {
+    uint4 a[kMergeRowsPerThread], bb[kMergeRowsPerThread];
+    float la[kMergeRowsPerThread], lb[kMergeRowsPerThread];
+    int li[kMergeRowsPerThread];
+    bool live[kMergeRowsPerThread];
+#pragma unroll
+    for (int u = 0; u < kMergeRowsPerThread; ++u) {
+      const int idx = ((it0 + u) << 5) + lane;  // < 2^31 (checked by the launcher)
+      live[u] = it0 + u < n_items && idx < n_vec;
+      const int row = idx >> vpr_log2;  // (b, s, h), h fastest
+      const int bs = row / H;
+      const int h = row - bs * H;
+      const int b = bs / S;
+      li[u] = (b * H + h) * S + (bs - b * S);
+      if (live[u]) {
+        a[u] = o_a[idx];
+        bb[u] = o_b[idx];
+        la[u] = lse_a[li[u]];
+        lb[u] = lse_b[li[u]];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kMergeRowsPerThread; ++u) {
+      if (!live[u]) continue;
+      const float mx = fmaxf(la[u], lb[u]);
+      float wa = 0.f, wb = 0.f, L = -INFINITY;
+      if (mx != -INFINITY) {
+        const float ea = expf(la[u] - mx), eb = expf(lb[u] - mx);
+        const float tot = ea + eb;
+        L = mx + logf(tot);
+        wa = ea / tot;
+        wb = eb / tot;
+      }
+      uint4 r;
+      if (kBf16) merge_vec_bf16(a[u], bb[u], wa, wb, r);
+      else merge_vec_f32(a[u], bb[u], wa, wb, r);
+      o[((it0 + u) << 5) + lane] = r;
+      if (leader) lse[li[u]] = L;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ split-KV combine
 // n partial results of the same queries over disjoint key ranges (split-KV), each a
 // normalised O (dtype of out) with its LSE, are folded exactly -- optionally together with
@@ -498,6 +554,25 @@ cudaError_t launch_merge(const void* o_a, const float* lse_a, const void* o_b, c
                          cudaStream_t stream) {
   const long long n_rows = (long long)B * S * H;
   const int vpr = D * elem_bytes / 16;  // 16-byte vectors per row (validated: 1..256)
+  const long long n_vec = n_rows * vpr;
+  if (vpr <= 32 && (vpr & (vpr - 1)) == 0 && n_vec <= 0x7fffffffLL - 32 * (kMergeRowsPerThread + 1)) {
+    int vpr_log2 = 0;
+    while ((1 << vpr_log2) < vpr) ++vpr_log2;
+    const long long items = (n_vec + 31) / 32;
+    const long long warps_needed = (items + kMergeRowsPerThread - 1) / kMergeRowsPerThread;
+    const long long blocks_needed = (warps_needed * 32 + kMergeThreads - 1) / kMergeThreads;
+    const long long cap = (long long)sm_count() * 4;  // all resident (64 registers a thread)
+    const unsigned blocks = unsigned(blocks_needed < cap ? blocks_needed : cap);
+    if (elem_bytes == 2)
+      merge_rows_kernel<true><<<blocks, kMergeThreads, 0, stream>>>(
+          static_cast<const uint4*>(o_a), lse_a, static_cast<const uint4*>(o_b), lse_b,
+          static_cast<uint4*>(o), lse, H, S, int(n_vec), vpr_log2);
+    else
+      merge_rows_kernel<false><<<blocks, kMergeThreads, 0, stream>>>(
+          static_cast<const uint4*>(o_a), lse_a, static_cast<const uint4*>(o_b), lse_b,
+          static_cast<uint4*>(o), lse, H, S, int(n_vec), vpr_log2);
+    return cudaGetLastError();
+  }
   const int rows_per_group = vpr >= kMergeThreads ? 1 : kMergeThreads / vpr;
   const long long rows_per_block = (long long)rows_per_group * kMergeRowsPerThread;
   const long long blocks = (n_rows + rows_per_block - 1) / rows_per_block;
