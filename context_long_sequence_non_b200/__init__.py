@@ -34,4 +34,4 @@ from ._binding import (  # noqa: F401
     status_str,
     version,
 )
-from .paths import ring_attention, ulysses_attention  # noqa: F401
+from .paths import UlyssesPlan, UlyssesStreamer, ring_attention, ulysses_attention  # noqa: F401

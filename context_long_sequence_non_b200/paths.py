@@ -111,3 +111,56 @@ def ulysses_attention(q_shards, k_shards, v_shards, P, scale=None, stream=None):
     plan = UlyssesPlan(P, S_l, H, D, dtype=q_shards.dtype, device=q_shards.device)
     out, lse = plan.run(q_shards, k_shards, v_shards, scale=scale, stream=stream)
     return out, lse
+
+
+class UlyssesStreamer:
+    """Host-to-host Ulysses passes with the copies of neighbouring steps overlapped with
+    compute.
+
+    ``depth`` device buffer sets rotate.  Step i's Q/K/V go host -> device on an upload
+    stream, its pass runs on the compute stream, and O and LSE go device -> host on a
+    download stream.  Events order the three per buffer set:
+    - upload i after the pass that last read set i % depth;
+    - pass i after upload i and after the download that last emptied the set's outputs;
+    - download i after pass i.
+
+    So the upload of step i+1 and the download of step i-1 run while step i computes.
+    Host buffers should be pinned, or the copies are not asynchronous.  ``submit`` returns
+    the event that completes when step i's outputs are on the host.
+    """
+
+    def __init__(self, P, S_local, H, D, dtype=torch.bfloat16, device="cuda", depth=2):
+        self.depth = depth
+        self.plans = [UlyssesPlan(P, S_local, H, D, dtype=dtype, device=device)
+                      for _ in range(depth)]
+        shard = (P, S_local, H, D)
+        self.inputs = [tuple(torch.empty(shard, dtype=dtype, device=device) for _ in range(3))
+                       for _ in range(depth)]
+        self.compute = torch.cuda.current_stream(device)
+        self.upload = torch.cuda.Stream(device)
+        self.download = torch.cuda.Stream(device)
+        ev = lambda: [torch.cuda.Event() for _ in range(depth)]
+        self.uploaded, self.computed, self.downloaded = ev(), ev(), ev()
+        self.step = 0
+
+    def submit(self, hq, hk, hv, h_out, h_lse, scale=None):
+        k = self.step % self.depth
+        plan, (dq, dk, dv) = self.plans[k], self.inputs[k]
+        # waiting on an event that was never recorded returns at once (first rotation)
+        self.upload.wait_event(self.computed[k])
+        with torch.cuda.stream(self.upload):
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            self.uploaded[k].record(self.upload)
+        self.compute.wait_event(self.uploaded[k])
+        self.compute.wait_event(self.downloaded[k])
+        plan.run(dq, dk, dv, scale=scale, stream=self.compute)
+        self.computed[k].record(self.compute)
+        self.download.wait_event(self.computed[k])
+        with torch.cuda.stream(self.download):
+            h_out.copy_(plan.out, non_blocking=True)
+            h_lse.copy_(plan.lse, non_blocking=True)
+            self.downloaded[k].record(self.download)
+        self.step += 1
+        return self.downloaded[k]

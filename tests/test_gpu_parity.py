@@ -485,3 +485,28 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     o, l = cp.fwd(q, k, v)
     torch.cuda.synchronize()
     check_o(o, ref.attention(q.cpu(), k.cpu(), v.cpu(), 1 / math.sqrt(128))[0], "bf16_out", "after")
+
+
+# ----------------------------------------------------------------------------- streaming
+
+
+def test_ulysses_streamer_matches_plan():
+    # host-to-host passes with overlapped copies: each step's outputs equal a plain
+    # UlyssesPlan pass on the same inputs, bit for bit, whatever the buffer rotation
+    P, S_l, H, D, steps = 2, 320, 4, 128, 5
+    g = torch.Generator().manual_seed(55)
+    host = [[W.randn((P, S_l, H, D), g, 1.0, "bf16").pin_memory() for _ in range(3)]
+            for _ in range(steps)]
+    outs = [(torch.empty((P, S_l, H, D), dtype=torch.bfloat16).pin_memory(),
+             torch.empty((P, H // P, P * S_l), dtype=torch.float32).pin_memory())
+            for _ in range(steps)]
+    st = cp.UlyssesStreamer(P, S_l, H, D, device=DEV, depth=2)
+    done = [st.submit(*host[i], *outs[i], scale=1 / math.sqrt(D)) for i in range(steps)]
+    done[-1].synchronize()
+    torch.cuda.synchronize()
+    plan = UlyssesPlan(P, S_l, H, D)
+    for i in range(steps):
+        o, l = plan.run(*(t.to(DEV) for t in host[i]), scale=1 / math.sqrt(D))
+        torch.cuda.synchronize()
+        assert torch.equal(bits(outs[i][0]), bits(o.cpu())), i
+        assert torch.equal(outs[i][1], l.cpu()), i
