@@ -224,11 +224,15 @@ __global__ void __launch_bounds__(kMergeThreads, 4) merge_rows_kernel(
       const float mx = fmaxf(la[u], lb[u]);
       float wa = 0.f, wb = 0.f, L = -INFINITY;
       if (mx != -INFINITY) {
-        const float ea = expf(la[u] - mx), eb = expf(lb[u] - mx);
+        // CUDA's fast intrinsics: the arguments are <= 0 and tot is in [1, 2], where their
+        // errors (a few float ulps) stay far below the merge's fp32 / LSE tolerances; every
+        // lane of a row computes the same weights
+        const float ea = __expf(la[u] - mx), eb = __expf(lb[u] - mx);
         const float tot = ea + eb;
-        L = mx + logf(tot);
-        wa = ea / tot;
-        wb = eb / tot;
+        const float inv = __fdividef(1.0f, tot);
+        L = mx + __logf(tot);
+        wa = ea * inv;
+        wb = eb * inv;
       }
       uint4 r;
       if (kBf16) merge_vec_bf16(a[u], bb[u], wa, wb, r);
