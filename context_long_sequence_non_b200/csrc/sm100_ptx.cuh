@@ -97,27 +97,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
-// As mbar_wait, but polling without a suspend-time hint: for a wait on the critical path
-// whose thread has nothing else to do and where the wake-up latency of a parked thread
-// matters more than the issue slots the polling takes.
-__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity,
-                                               volatile int* abort_flag, int* err,
-                                               long long limit) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (clock64() - t0 > limit) {
-      *abort_flag = 1;
-      atomicOr(err, kDevErrTimeout);
-      return false;
-    }
-  }
-}
-
 // Bounded wait used only on the way out of a kernel (never raises the abort flag): gives
 // in-flight asynchronous copies or MMAs up to `limit` cycles to land before the CTA's
 // shared and tensor memory are released.
