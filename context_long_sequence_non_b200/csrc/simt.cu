@@ -378,22 +378,29 @@ __device__ __forceinline__ uint4 rms_normalise(uint4 in, bool live, int row_vec,
     f[2 * t] = live ? __uint_as_float(w[t] << 16) : 0.f;  // bf16 -> fp32 is exact
     f[2 * t + 1] = live ? __uint_as_float(w[t] & 0xFFFF0000u) : 0.f;
   }
-  float ss = 0.f;
+  // packed fp32x2 arithmetic: per lane the same IEEE operations as the scalar forms, in
+  // half the issue slots (the fused permute is issue-bound)
+  float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+  for (int e = 0; e < 8; e += 2) {
+    const float2 fe = make_float2(f[e], f[e + 1]);
+    ss2 = ffma2(fe, fe, ss2);
+  }
+  float ss = ss2.x + ss2.y;
   for (int o = 1; o < row_vec; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   const float a = ss * inv_d + eps;
   const float r = a > 0.f ? rsqrt_refined(a) : 0.f;  // an all-zero row with eps = 0 stays 0
   if (!live) return in;
-  float y[8];
+  const float2 r2 = make_float2(r, r), s2 = make_float2(out_scale, out_scale);
+  uint32_t w_out[4];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) y[e] = (f[e] * r) * g[e];
-  if (out_scale != 1.0f) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) y[e] *= out_scale;
+  for (int t = 0; t < 4; ++t) {
+    float2 y = fmul2(fmul2(make_float2(f[2 * t], f[2 * t + 1]), r2),
+                     make_float2(g[2 * t], g[2 * t + 1]));
+    if (out_scale != 1.0f) y = fmul2(y, s2);
+    w_out[t] = pack_bf16x2(y.x, y.y);
   }
-  return make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                    pack_bf16x2(y[6], y[7]));
+  return make_uint4(w_out[0], w_out[1], w_out[2], w_out[3]);
 }
 
 template <bool kToHead, bool kNorm>
