@@ -335,6 +335,10 @@ constexpr int kPermUnroll = 4;
 struct PermuteSet {
   const uint4* src[3];
   uint4* dst[3];
+  // blocks [block_begin[t], block_begin[t + 1]) of the 1-D grid serve tensor t; the split
+  // follows each tensor's work (a normalised tensor costs about twice a plain copy), so
+  // all tensors finish together
+  int block_begin[4];
 };
 
 // Optional RMSNorm of every head row on the way through (the Q/K norm of the
@@ -404,17 +408,21 @@ __device__ __forceinline__ uint4 rms_normalise(uint4 in, bool live, int row_vec,
 }
 
 template <bool kToHead, bool kNorm>
-__global__ void __launch_bounds__(kPermThreads, kNorm ? 5 : 1) permute_kernel(const __grid_constant__ PermuteSet set,
+__global__ void __launch_bounds__(kPermThreads, 5) permute_kernel(const __grid_constant__ PermuteSet set,
                                                                 const __grid_constant__ RowNorm nrm,
                                                                 int P, int S_l, int run_vec,
                                                                 int chunks, int n_items) {
   // blockIdx.y picks the tensor (uniform per block); item = (dst row, 32-vector chunk)
-  const uint4* __restrict__ src = set.src[blockIdx.y];
-  uint4* __restrict__ dst = set.dst[blockIdx.y];
+  const int bx = int(blockIdx.x);
+  const int tsr = int(bx >= set.block_begin[1]) + int(bx >= set.block_begin[2]);  // tensor
+  const int local_block = bx - set.block_begin[tsr];
+  const int n_blocks = set.block_begin[tsr + 1] - set.block_begin[tsr];
+  const uint4* __restrict__ src = set.src[tsr];
+  uint4* __restrict__ dst = set.dst[tsr];
   const int lane = threadIdx.x & 31;
-  const int warp = int((blockIdx.x * kPermThreads + threadIdx.x) >> 5);
-  const int n_warps = int((gridDim.x * kPermThreads) >> 5);
-  const float* __restrict__ gamma = kNorm ? nrm.gamma[blockIdx.y] : nullptr;  // per block
+  const int warp = (local_block * kPermThreads + int(threadIdx.x)) >> 5;
+  const int n_warps = (n_blocks * kPermThreads) >> 5;
+  const float* __restrict__ gamma = kNorm ? nrm.gamma[tsr] : nullptr;  // per block
   float g[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (kNorm && gamma != nullptr) load_gamma8(gamma, (lane % nrm.row_vec) * 8, g);
   for (int it0 = warp * kPermUnroll; it0 < n_items; it0 += n_warps * kPermUnroll) {
@@ -644,9 +652,24 @@ static cudaError_t launch_permute(bool to_head, const void* const* src, void* co
   if (n_items > 0x7fffffffLL) return cudaErrorInvalidValue;  // 32-bit item index
   const long long warps_needed = (n_items + kPermUnroll - 1) / kPermUnroll;
   const long long blocks_needed = (warps_needed * 32 + kPermThreads - 1) / kPermThreads;
-  const long long cap = (long long)sm_count() * 8 / n_tensors + 1;
-  const long long blocks = blocks_needed < cap ? blocks_needed : cap;
-  const dim3 grid{unsigned(blocks), unsigned(n_tensors), 1u};
+  // about 8 resident blocks per SM in total, shared out by each tensor's cost
+  int weight[3] = {0, 0, 0}, weight_sum = 0;
+  for (int t = 0; t < n_tensors; ++t) {
+    weight[t] = (nrm != nullptr && nrm->gamma[t] != nullptr) ? 2 : 1;
+    weight_sum += weight[t];
+  }
+  const long long total = (long long)sm_count() * 8;
+  set.block_begin[0] = 0;
+  for (int t = 0; t < 3; ++t) {
+    long long b = 0;
+    if (t < n_tensors) {
+      b = total * weight[t] / weight_sum;
+      if (b > blocks_needed) b = blocks_needed;
+      if (b < 1) b = 1;
+    }
+    set.block_begin[t + 1] = set.block_begin[t] + int(b);
+  }
+  const dim3 grid{unsigned(set.block_begin[3]), 1u, 1u};
   const RowNorm none{};
   if (nrm != nullptr)
     permute_kernel<true, true><<<grid, kPermThreads, 0, stream>>>(set, *nrm, P, S_local,
