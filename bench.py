@@ -24,6 +24,7 @@ import os
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 import torch
@@ -104,7 +105,11 @@ def aggregate(dist, elapsed_ms: float, units: float, device=None):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 50 ms during the timed region."""
+    """nvidia-smi clocks and throttle reasons sampled every 50 ms during the timed region.
+
+    nvidia-smi can take a second or more to print its first sample, so its output is read
+    on a thread and ``start`` returns only once the first sample has arrived (or after
+    ``wait_s``): the timed region that follows is then covered from its first moment."""
 
     FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -112,8 +117,13 @@ class ClockSampler:
 
     def __init__(self, gpu_index: int, path: str | None = None):
         self.gpu_index, self.proc, self.path = gpu_index, None, path
+        self.lines, self.reader = [], None
 
-    def start(self):
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line)
+
+    def start(self, wait_s: float = 10.0):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}",
@@ -121,42 +131,57 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+            return
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+        t0 = time.time()
+        while not self.lines and time.time() - t0 < wait_s and self.proc.poll() is None:
+            time.sleep(0.02)
 
     def stop(self, t_begin: float | None = None, t_end: float | None = None):
-        """Stop sampling; summarise the samples taken inside [t_begin, t_end] (epoch s)."""
+        """Stop sampling; summarise the samples taken inside [t_begin, t_end] (epoch s), or
+        the ones nearest to it (within 1 s) when the region was too short to catch one."""
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)  # one more sample after the region
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-            out, _ = self.proc.communicate()
-        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+            self.proc.wait()
+        if self.reader is not None:
+            self.reader.join(timeout=5)
+        out = "".join(self.lines)
         if self.path:
             with open(self.path, "w") as f:
                 f.write(out)
         import datetime
 
-        sm, mx, reasons, power = [], None, set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
+        parsed = []
+        for r in (r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8):
             try:
                 ts = datetime.datetime.strptime(r[0].strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
-                if t_begin is not None and not (t_begin <= ts <= t_end):
-                    continue
-                sm.append(float(r[1]))
-                mx = float(r[2])
-                power.append(float(r[3]))
+                parsed.append((ts, float(r[1]), float(r[2]), float(r[3]),
+                               [n for n, val in zip(names, r[5:9])
+                                if val.strip().lower() == "active"]))
             except ValueError:
                 continue
-            for n, val in zip(names, r[5:9]):
-                if val.strip().lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "sm_mhz_min": min(sm) if sm else None, "reasons": sorted(reasons),
-                "samples": len(sm), "power_w_max": max(power) if power else None,
-                "window": "samples inside the timed region"}
+        window = "samples inside the timed region"
+        chosen = parsed
+        if t_begin is not None:
+            chosen = [x for x in parsed if t_begin <= x[0] <= t_end]
+            if not chosen:
+                chosen = [x for x in parsed if t_begin - 1.0 <= x[0] <= t_end + 1.0]
+                window = "samples within 1 s of the timed region (none inside it)"
+        sm = [x[1] for x in chosen]
+        reasons = sorted({n for x in chosen for n in x[4]})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": chosen[-1][2] if chosen else None,
+                "sm_mhz_min": min(sm) if sm else None, "reasons": reasons,
+                "samples": len(sm), "power_w_max": max(x[3] for x in chosen) if chosen else None,
+                "window": window}
 
 
 # --------------------------------------------------------------------------- peaks
@@ -227,8 +252,7 @@ def run_ours(args, world, rank, local):
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    clocks.start()
-    time.sleep(0.3)  # let the sampler take its first readings
+    clocks.start()  # returns once nvidia-smi is reporting
     wall0 = time.time()
     t0.record(stream)
     for i in range(args.steps):
