@@ -244,8 +244,8 @@ def run_ours(args, world, rank, local):
     if Bd.device_error() != 0:
         raise RuntimeError("bounded wait ran out during warm-up")
 
-    clocks = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
-                          if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else None)
+    clocks = ClockSampler(local, args.clocks_csv.replace("{rank}", str(rank))
+                          if args.clocks_csv else None)
     attn_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                    for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -622,6 +622,9 @@ def main(argv=None):
     ap.add_argument("--profile", action="store_true",
                     help="for profiler captures: run only warm-up + timed steps (no aux "
                          "kernels, no end-to-end pass, no CPU baseline)")
+    ap.add_argument("--clocks-csv", default=None, metavar="PATH",
+                    help="also write the raw nvidia-smi samples of the timed region to PATH "
+                         "('{rank}' is replaced by the rank)")
     ap.add_argument("--qk-norm", action="store_true",
                     help="step variant: Q/K RMSNorm fused into one Q/K/V seq2head launch "
                          "(not the headline step; for profiling that kernel)")
