@@ -126,10 +126,14 @@ class UlyssesStreamer:
 
     So the upload of step i+1 and the download of step i-1 run while step i computes.
     Host buffers should be pinned, or the copies are not asynchronous.  ``submit`` returns
-    the event that completes when step i's outputs are on the host.
+    the event that completes when step i's outputs are on the host.  The copies are
+    asynchronous: a step's host inputs must not be modified, and its host outputs not
+    read or reused, until that event has completed.
     """
 
     def __init__(self, P, S_local, H, D, dtype=torch.bfloat16, device="cuda", depth=2):
+        if depth < 1:
+            raise ValueError("depth must be at least 1 (2 or more to overlap copies)")
         self.depth = depth
         self.plans = [UlyssesPlan(P, S_local, H, D, dtype=dtype, device=device)
                       for _ in range(depth)]
