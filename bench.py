@@ -38,16 +38,56 @@ from context_long_sequence_non_b200 import workloads as W  # noqa: E402
 METRIC = "non-causal bf16 attention TFLOPS at S=44160 on 1 B200; % of dense BF16 peak"
 UNIT = "TFLOP/s"
 WORKLOAD = W.WORKLOADS[4]
-# DRAM bytes (read + write) per launch of the attention kernel on this workload, from the
-# ncu capture summarised in profiles/attn_fwd_sm100_ulysses_s44160.md; valid only for the
-# kernel version named there (set to None whenever the kernel changes until re-captured).
-ATTN_TRAFFIC_BYTES = 597_763_840 + 168_522_496
+# DRAM bytes (read + write) per launch of each attention kernel on this workload, from one
+# ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the kernel and by the
+# SHA-256 of the kernel sources the capture was taken with.  When the sources hash to
+# something else the figure no longer describes the kernel that runs, and the line reports
+# traffic null until a new capture is recorded here.
+ATTN_SOURCES = ("context_long_sequence_non_b200/csrc/attn_sm100.cu",
+                "context_long_sequence_non_b200/csrc/sm100_ptx.cuh")
+ATTN_TRAFFIC = {
+    "attn_fwd_sm100_kernel<128,0,0>": {
+        "sources_sha256": "670a6a10557d5e93274985aea76ef3e33e3c4bdecf726c251274211068314865",
+        "bytes": 597_763_840 + 168_522_496,
+    },
+}
 L2_NOTE = ("inputs larger than L2: each step streams 543 MB of Q/K/V shards plus 724 MB of "
            "permute traffic through the 126 MB L2")
 
 
-def workload_config(qk_norm=False):
+def attn_sources_sha256():
+    import hashlib
+
+    h = hashlib.sha256()
+    for rel in ATTN_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def attn_traffic(kernel):
+    """ncu DRAM bytes per launch for ``kernel``, or None when no capture matches its
+    current sources."""
+    rec = ATTN_TRAFFIC.get(kernel)
+    if rec is None or rec["sources_sha256"] != attn_sources_sha256():
+        return None
+    return rec["bytes"]
+
+
+def workload_config(qk_norm=False, step="fused"):
     w = WORKLOAD
+    if step == "fused":
+        return {
+            "workload": ("ulysses-cp8-s44160: P=8 virtual ranks x [5520 tokens][16 heads][128] "
+                         "bf16 Q/K/V shards in, O shards + fp32 LSE out; the Ulysses re-partitions "
+                         "(seq2head of Q/K/V, head2seq of O) done by the attention kernel's own "
+                         "addressing (one kernel: non-causal attention over 8 head groups x 2 "
+                         "heads, S=44160, D=128, fp32 accumulate, bf16 O); bit-identical to the "
+                         "3x seq2head + attention + head2seq launches"),
+            "B": w.B, "H": w.H, "S": w.Sq, "D": w.D, "P": w.P, "step": "fused",
+            "inputs": "iid N(0,1), torch.Generator seed 4000, rounded to bf16",
+            "l2": L2_NOTE,
+        }
     if qk_norm:
         return {
             "workload": ("ulysses-cp8-s44160 with Q/K RMSNorm: P=8 virtual ranks x [5520 tokens]"
@@ -62,7 +102,7 @@ def workload_config(qk_norm=False):
         "workload": (f"ulysses-cp8-s44160: P=8 virtual ranks x [5520 tokens][16 heads][128] bf16 "
                      f"Q/K/V, 3x seq2head + non-causal attention (8 head groups x 2 heads, "
                      f"S=44160, D=128, fp32 accumulate, bf16 O + fp32 LSE) + head2seq"),
-        "B": w.B, "H": w.H, "S": w.Sq, "D": w.D, "P": w.P,
+        "B": w.B, "H": w.H, "S": w.Sq, "D": w.D, "P": w.P, "step": "plain",
         "inputs": "iid N(0,1), torch.Generator seed 4000, rounded to bf16",
         "l2": L2_NOTE,
     }
@@ -219,12 +259,11 @@ def run_ours(args, world, rank, local):
     plan = UlyssesPlan(P, S_l, H, w.D, device=dev)
     stream = torch.cuda.current_stream(dev)
     flops = w.attn_flops
-    launches_per_step = 3 if args.qk_norm else 5
     if args.qk_norm:  # the sample's Q/K RMSNorm fused into one Q/K/V seq2head launch
         gq = W.norm_weights(w.D, seed=41).to(dev)
         gk = W.norm_weights(w.D, seed=42).to(dev)
 
-    def step(ev_attn=None):
+    def plain_step(ev_attn=None):
         if args.qk_norm:
             cp.seq2head_qkv_norm(q, k, v, P, gq, gk, out=(plan.qh, plan.kh, plan.vh))
         else:
@@ -238,37 +277,75 @@ def run_ours(args, world, rank, local):
             ev_attn[1].record(stream)
         cp.head2seq(plan.oh, P, out=plan.out)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    if Bd.device_error() != 0:
-        raise RuntimeError("bounded wait ran out during warm-up")
+    def fused_step(ev_attn=None):
+        # sharded Q/K/V in, sharded O + LSE out: the same work and the same bits as
+        # plain_step, the re-partitions done by the attention kernel's addressing
+        if ev_attn is not None:
+            ev_attn[0].record(stream)
+        cp.ulysses_fwd(q, k, v, P, out=plan.out, lse=plan.lse, scale=w.softmax_scale)
+        if ev_attn is not None:
+            ev_attn[1].record(stream)
 
-    clocks = ClockSampler(local, args.clocks_csv.replace("{rank}", str(rank))
-                          if args.clocks_csv else None)
-    attn_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    clocks.start()  # returns once nvidia-smi is reporting
-    wall0 = time.time()
-    t0.record(stream)
-    for i in range(args.steps):
-        step(attn_events[i])
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
-    wall1 = time.time()
-    clk = clocks.stop(wall0, wall1)
-    if dist is not None:
-        dist.barrier()
-    elapsed_ms = t0.elapsed_time(t1)
-    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in attn_events)
-    if Bd.device_error() != 0:
-        raise RuntimeError("bounded wait ran out during the timed region")
-    max_ms, total_flops = aggregate(dist, elapsed_ms, flops * args.steps,
-                                    device=dev if dist is not None else None)
+    def timed_steps(step, tag):
+        """W untimed warm-up steps, then exactly K timed steps bracketed by a barrier and a
+        device synchronize on both sides; CUDA events on the launching stream around the
+        whole region and around each attention launch; clocks sampled during it."""
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize(dev)
+        if Bd.device_error() != 0:
+            raise RuntimeError(f"bounded wait ran out during the {tag} warm-up")
+        path = (args.clocks_csv.replace("{rank}", str(rank)).replace("{step}", tag)
+                if args.clocks_csv else None)
+        clocks = ClockSampler(local, path)
+        attn_events = [(torch.cuda.Event(enable_timing=True),
+                        torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        clocks.start()  # returns once nvidia-smi is reporting
+        wall0 = time.time()
+        t0.record(stream)
+        for i in range(args.steps):
+            step(attn_events[i])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        wall1 = time.time()
+        clk = clocks.stop(wall0, wall1)
+        if dist is not None:
+            dist.barrier()
+        elapsed_ms = t0.elapsed_time(t1)
+        attn_ms = statistics.mean(a.elapsed_time(b) for a, b in attn_events)
+        if Bd.device_error() != 0:
+            raise RuntimeError(f"bounded wait ran out during the {tag} timed region")
+        max_ms, total_flops = aggregate(dist, elapsed_ms, flops * args.steps,
+                                        device=dev if dist is not None else None)
+        return max_ms, total_flops, attn_ms, clk
+
+    peaks = measured_peaks()
+    variants = {
+        "fused": (fused_step, 1, "attn_fwd_sm100_kernel<128,0,2>",
+                  "cpattn_ulysses_fwd: one kernel, sharded Q/K/V in, sharded O + LSE out"),
+        "plain": (plain_step, 3 if args.qk_norm else 5, "attn_fwd_sm100_kernel<128,0,0>",
+                  ("seq2head_qkv_norm + cpattn_fwd + head2seq" if args.qk_norm else
+                   "3x cpattn_seq2head + cpattn_fwd + cpattn_head2seq")),
+    }
+    head = "plain" if args.qk_norm else args.step
+    # profiler runs time the headline variant only, so a launch list holds one step kind
+    order = [head] + [n for n in variants
+                      if n != head and not args.qk_norm and not args.profile]
+    results = {}
+    for name in order:
+        fn, launches, kernel, what = variants[name]
+        max_ms, total_flops, attn_ms, clk = timed_steps(fn, name)
+        value = total_flops / (max_ms * 1e-3) / 1e12
+        results[name] = {"value": round(value, 2), "unit": UNIT,
+                         "ms_per_step": round(max_ms / args.steps, 4),
+                         "attn_kernel": kernel, "attn_ms": round(attn_ms, 4),
+                         "attn_TFLOP/s": round(flops / (attn_ms * 1e-3) / 1e12, 2),
+                         "gpu_launches": launches * args.steps, "what": what, "clocks": clk,
+                         "_raw": (max_ms, total_flops, attn_ms)}
 
     if args.profile:  # profiler runs: the timed steps only, nothing else launched
         aux, e2e = None, None
@@ -279,35 +356,43 @@ def run_ours(args, world, rank, local):
         # ---- end to end through the public API with host buffers
         e2e = e2e_run(cp, UlyssesPlan, w, x, dev, stream, args)
 
-    peaks = measured_peaks()
+    hr = results[head]
+    max_ms, total_flops, attn_ms = hr.pop("_raw")
+    for r in results.values():
+        r.pop("_raw", None)
     value = total_flops / (max_ms * 1e-3) / 1e12
     achieved = flops / (attn_ms * 1e-3) / 1e12
     long_run = max_ms > 1000.0
     peak = peaks["bf16_tflops_sustained"] if long_run else peaks["bf16_tflops"]
+    kernel = hr["attn_kernel"]
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(max_ms / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(args.qk_norm),
+        "config": workload_config(args.qk_norm, head),
         "frac_of_dense_bf16_peak": round(value / peak, 4),
         "roofline": {
-            "bound": "tensor", "kernel": "attn_fwd_sm100_kernel<128,false>",
+            "bound": "tensor", "kernel": kernel,
             "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4),
             "peak_kind": (f"{peaks['source']} cuBLAS bf16 "
                           f"{'sustained' if long_run else 'burst'}"),
             "algorithmic_flops_per_launch": flops,
-            "avg_launch_ms": round(attn_ms, 4), "traffic": ATTN_TRAFFIC_BYTES,
+            "avg_launch_ms": round(attn_ms, 4), "traffic": attn_traffic(kernel),
             "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
+            "traffic_source": ("ncu capture of this kernel, recorded with the SHA-256 of its "
+                               "sources; null when the sources have changed since"),
+            "sources_sha256": attn_sources_sha256(),
             # Q, K, V read once and O written once (four equal bf16 tensors) + fp32 LSE
             "algorithmic_bytes_per_launch": 4 * q.numel() * q.element_size()
             + plan.lse.numel() * 4,
         },
+        "step_variants": results,
         "aux": aux,
         "e2e": e2e,
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk,
+        "gpu_launches": hr["gpu_launches"],
+        "clocks": hr["clocks"],
     }
     if rank == 0 and world == 1 and not (args.no_cpu_baseline or args.profile):
         line["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)
@@ -536,6 +621,12 @@ def e2e_run(cp, UlyssesPlan, w, x, dev, stream, args):
 # --------------------------------------------------------------------------- CPU oracle
 
 
+# Query rows per oracle sample, for the CPU baseline and the reference arm alike: about
+# 128 rows per head, so each head's products are real matrix products (a handful of rows
+# per head would time BLAS at matrix-vector efficiency and understate the oracle).
+ORACLE_ROWS = 2048
+
+
 def oracle_sample(n_rows, seed):
     """The fp64 oracle on ``n_rows`` sampled query rows of the Ulysses workload (each row
     attends over all 44160 keys of its head).  Returns (seconds, flops, cores)."""
@@ -566,32 +657,32 @@ def _oracle_inputs():
     return _INPUTS
 
 
+def _sample_text(rows, spent):
+    return (f"{rows} query rows of the S=44160 Ulysses workload in samples of {ORACLE_ROWS} "
+            f"(~{ORACLE_ROWS // 16} per head), each row over all 44160 keys, fp64 NumPy/BLAS, "
+            f"{spent:.1f} s")
+
+
 def cpu_baseline(budget_s=15.0):
-    n, spent, flops, cores = 64, 0.0, 0.0, 1
-    rounds = 0
-    while spent < budget_s and rounds < 12:
-        dt, f, cores = oracle_sample(n, seed=100 + rounds)
+    oracle_sample(ORACLE_ROWS // 8, seed=99)  # untimed: BLAS threads and page-in
+    spent, flops, cores, rounds = 0.0, 0.0, 1, 0
+    while spent < budget_s and rounds < 40:
+        dt, f, cores = oracle_sample(ORACLE_ROWS, seed=100 + rounds)
         spent += dt
         flops += f
         rounds += 1
-        if dt < budget_s / 4:
-            n *= 2
     return {"value": round(flops / spent / 1e12, 6), "unit": UNIT, "cores": cores,
-            "kind": "oracle",
-            "sample": (f"{int(flops / (4 * WORKLOAD.Skv * WORKLOAD.D))} query rows of the "
-                       f"S=44160 Ulysses workload (each over all 44160 keys), fp64 NumPy/BLAS, "
-                       f"{spent:.1f} s")}
+            "kind": "oracle", "sample": _sample_text(rounds * ORACLE_ROWS, spent)}
 
 
 def run_reference(args, world, rank):
     if rank != 0:
         return  # the CPU oracle arm runs on rank 0 only
-    rows_per_step = 128
     for i in range(args.warmup):
-        oracle_sample(rows_per_step, seed=1 + i)
+        oracle_sample(ORACLE_ROWS // 8, seed=1 + i)
     tot_t, tot_f, cores = 0.0, 0.0, 1
     for i in range(args.steps):
-        dt, f, cores = oracle_sample(rows_per_step, seed=1000 + i)
+        dt, f, cores = oracle_sample(ORACLE_ROWS, seed=1000 + i)
         tot_t += dt
         tot_f += f
     value = tot_f / tot_t / 1e12
@@ -600,11 +691,10 @@ def run_reference(args, world, rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(tot_t / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(),
+        "config": workload_config(step=args.step),
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores,
                          "kind": "oracle",
-                         "sample": f"{rows_per_step} query rows per step of the S=44160 Ulysses "
-                                   f"workload, each over all 44160 keys, fp64 NumPy/BLAS"},
+                         "sample": "one step = " + _sample_text(ORACLE_ROWS, tot_t / args.steps)},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -623,11 +713,15 @@ def main(argv=None):
                     help="for profiler captures: run only warm-up + timed steps (no aux "
                          "kernels, no end-to-end pass, no CPU baseline)")
     ap.add_argument("--clocks-csv", default=None, metavar="PATH",
-                    help="also write the raw nvidia-smi samples of the timed region to PATH "
-                         "('{rank}' is replaced by the rank)")
+                    help="also write the raw nvidia-smi samples of each timed region to PATH "
+                         "('{rank}' and '{step}' are replaced by the rank and step variant)")
     ap.add_argument("--qk-norm", action="store_true",
                     help="step variant: Q/K RMSNorm fused into one Q/K/V seq2head launch "
                          "(not the headline step; for profiling that kernel)")
+    ap.add_argument("--step", choices=("fused", "plain"), default="fused",
+                    help="the headline step: 'fused' = the Ulysses pass as one kernel "
+                         "(cpattn_ulysses_fwd), 'plain' = 3x seq2head + attention + head2seq; "
+                         "the other variant is timed the same way and reported beside it")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")

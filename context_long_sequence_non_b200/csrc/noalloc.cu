@@ -27,6 +27,9 @@ constexpr int kMaxDevices = 64;
 // g_noalloc_scratch is only a host-side stand-in for the symbol, never a device address, so
 // it is looked up with cudaGetSymbolAddress -- once per device, with that device current,
 // on the first call made on it -- and only the looked-up pointer is handed to kernels.
+// Under CUDA's lazy module loading (the default) this first lookup is also what loads the
+// module holding the array, so the first call on a device may reserve its 64 MiB and
+// synchronize; later calls only read the cached pointer.
 void* scratch_on_current_device(int* status) {
   static void* addr[kMaxDevices] = {nullptr};
   static std::mutex mu;
@@ -59,8 +62,16 @@ int cpattn_fwd_split_noalloc(const void* q, const void* k, const void* v, void* 
                              int B, int H, int Sq, int Skv, int D, float scale, int out_dtype,
                              int accumulate, int n_split, cpattn_stream_t stream) {
   // The size check comes first and needs no CUDA call: a request whose partials do not fit
-  // in the fixed scratch is refused before anything is set up or launched.
-  if (cpattn_fwd_split_workspace(B, H, Sq, D, n_split, out_dtype) > kNoAllocScratchBytes)
+  // in the fixed scratch is refused before anything is set up or launched.  It is made for
+  // the split count cpattn_fwd_split will actually use: that call lowers n_split to the
+  // number of 128-key blocks (every range holds at least one), so a request such as
+  // n_split = 8 over 256 keys needs the scratch of two ranges, not eight.
+  int n_used = n_split;
+  if (n_split >= 1 && Skv >= 0) {
+    const int n_kv = (Skv + 127) / 128;
+    if (n_used > n_kv) n_used = n_kv > 0 ? n_kv : 1;
+  }
+  if (cpattn_fwd_split_workspace(B, H, Sq, D, n_used, out_dtype) > kNoAllocScratchBytes)
     return CPATTN_ERR_SHAPE;
   int status = CPATTN_OK;
   void* scratch = scratch_on_current_device(&status);

@@ -186,8 +186,9 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
 // Rows of at most 32 vectors (bf16 D <= 256, fp32 D <= 128; vpr a power of two): warps
 // stride over items of 32 consecutive vectors = 32/vpr whole rows, kMergeRowsPerThread items
 // in flight, the grid a fixed multiple of the SM count (no tail wave).  A row's lanes all
-// sit in one warp, so an in-place LSE update needs no block barrier: the row's leader lane
-// writes L after, and from, the loads every lane of the warp issued first.
+// sit in one warp, so an in-place LSE update needs no block barrier, only a warp one: the
+// __syncwarp() between the load loop and the store loop orders every lane's read of
+// lse_a before the row leader's write of lse (which may be the same array).
 template <bool kBf16>
 __global__ void __launch_bounds__(kMergeThreads, 4) merge_rows_kernel(
     const uint4* o_a, const float* lse_a, const uint4* o_b, const float* lse_b, uint4* o,
@@ -218,6 +219,7 @@ __global__ void __launch_bounds__(kMergeThreads, 4) merge_rows_kernel(
         lb[u] = lse_b[li[u]];
       }
     }
+    __syncwarp();  // every lane's LSE reads above precede the leaders' LSE writes below
 #pragma unroll
     for (int u = 0; u < kMergeRowsPerThread; ++u) {
       if (!live[u]) continue;

@@ -132,7 +132,12 @@ CPATTN_API int cpattn_split_suggest(int B, int H, int Sq, int Skv);
  * until the process exits.  The call itself allocates nothing: it makes no cudaMalloc,
  * cudaFree or other allocating call.
  * The first call on a device looks up that device's address of the array (with the device
- * current); make that first call before any stream capture.
+ * current); make that first call before any stream capture.  Under CUDA's lazy module
+ * loading (the default) that first call is also when the array's module is loaded, so it
+ * may reserve the 64 MiB and synchronize the device: a caller that needs an
+ * allocation-free loop makes one warm-up call first.
+ * n_split is lowered exactly as cpattn_fwd_split lowers it (to the number of 128-key
+ * blocks), and the size check uses the lowered count.
  * All calls on a device share the one array and it keeps the last call's contents (each
  * call writes every byte it reads first, so nothing needs clearing): calls that overlap on
  * the GPU -- on different streams, or from different threads -- race on it and must not
@@ -239,7 +244,10 @@ CPATTN_API int cpattn_seq2head_qkv(const void* q, const void* k, const void* v, 
  * 推理实战", section 模型的核心结构): after Q and K are split into heads, every head row
  * is normalised in fp32 as x * rsqrt(mean(x^2) + eps) (eps = 1e-6 there), multiplied by a
  * weight and cast back to 16 bits.  For each of `rows` head rows of D elements:
- *   r = 1 / sqrt(sum_d x[d]^2 / D + eps)                  (fp32, IEEE sqrt and division)
+ *   r = 1 / sqrt(sum_d x[d]^2 / D + eps)                  (fp32: the hardware reciprocal
+ *                                                           square-root estimate refined by
+ *                                                           one Newton step, about an ulp of
+ *                                                           the correctly rounded value)
  *   y[d] = bf16_rne(((x[d] * r) * gamma[d]) * out_scale)  (fp32 products)
  * `out_scale` is the sample's split scale sqrt(sqrt(1/D)) when the caller keeps Q and K
  * pre-scaled (then pass scale = 1 to cpattn_fwd); pass 1 to apply 1/sqrt(D) to the

@@ -396,3 +396,58 @@ def test_planted_permute_mistake_is_caught(mistake):
 
     with pytest.raises(AssertionError):
         check_permute_golden(bad_seq2head, ref.head2seq)
+
+
+# ----------------------------------------------------------------------------- ring attention
+
+
+def check_ring_attention(ring_attention, seed):
+    """ring_attention over any split of the keys into chunks (empty, size-1, uneven) equals
+    attention over the concatenated chunks: against the loop-only brute force (independent
+    of ref.attention) and, for the closed form, a chunk repeated gives LSE + ln 2."""
+    r = _rng(60 + seed)
+    skv = int(r.integers(2, 24))
+    q, k, v = _rand(70 + seed, 1, 5, skv, 2, 3, sigma=1.3)
+    cuts = _split_points(skv, r)
+    if seed == 0:
+        cuts = [0, 1, 1, skv - 1, skv]  # size-1, empty, the bulk, size-1 tail
+    kc = [k[:, a:b] for a, b in zip(cuts, cuts[1:])]
+    vc = [v[:, a:b] for a, b in zip(cuts, cuts[1:])]
+    o, lse = ring_attention(q, kc, vc, 0.45)
+    ob, lb = brute.attention(q, k, v, 0.45)
+    np.testing.assert_allclose(o, np.asarray(ob), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, np.asarray(lb), rtol=1e-13, atol=1e-13)
+    # every chunk twice: the key multiset doubles, so O is unchanged and LSE gains ln 2
+    o2, l2 = ring_attention(q, kc + kc, vc + vc, 0.45)
+    np.testing.assert_allclose(o2, np.asarray(ob), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(l2, np.asarray(lb) + math.log(2), rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_ring_attention_equals_attention_over_concatenated_chunks(seed):
+    check_ring_attention(ref.ring_attention, seed)
+
+
+@pytest.mark.parametrize("mistake", ["drop_last_chunk", "kv_misaligned", "first_chunk_twice",
+                                     "unmerged_last"])
+def test_planted_ring_attention_mistake_is_caught(mistake):
+    def bad_ring(q, k_chunks, v_chunks, scale):
+        kc, vc = list(k_chunks), list(v_chunks)
+        if mistake == "drop_last_chunk":  # an off-by-one in the ring loop
+            kc, vc = kc[:-1], vc[:-1]
+        elif mistake == "kv_misaligned":  # V of the previous chunk paired with K
+            vc = vc[-1:] + vc[:-1]
+        elif mistake == "first_chunk_twice":
+            kc, vc = kc[:1] + kc, vc[:1] + vc
+        parts = [ref.attention(q, a, b, scale) for a, b in zip(kc, vc)]
+        if mistake == "unmerged_last":  # the last partial overwrites the running result
+            return parts[-1]
+        return ref.merge_chunks(parts)
+
+    caught = 0
+    for seed in range(5):
+        try:
+            check_ring_attention(bad_ring, seed)
+        except AssertionError:
+            caught += 1
+    assert caught >= 1, f"no pin caught the planted mistake {mistake!r}"

@@ -3,8 +3,11 @@ allocate device memory (its partials live in a fixed scratch array inside the li
 
 Called through the C ABI with ctypes and checked against cpattn_fwd_split given a
 caller-allocated workspace, on two calls in a row: a plain pass, then an accumulating pass
-that reuses the scratch the first call left behind.  Collected last so that a run stopping
-at the first failure has already run every other test; it also passes on its own.
+that reuses the scratch the first call left behind.  Both entry points run the same
+kernels on the same data with the same partial layout, so their results must be identical
+bit for bit.  After a warm-up call, a further call must leave the device's free memory
+unchanged (it allocates nothing).  Collected last so that a run stopping at the first
+failure has already run every other test; it also passes on its own.
 """
 
 import ctypes
@@ -46,18 +49,32 @@ def _p(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
+# (B, H, Sq, Skv, D, n_split requested, n_split the call uses)
+CASES = [
+    (1, 8, 300, 5000, 128, 4, 4),
+    (2, 3, 257, 1300, 64, 3, 3),  # D = 64, ragged query tail
+    # 8 ranges over 256 keys would need 65 MiB of partials; the call lowers the split to
+    # the two 128-key blocks there are, and two ranges fit in the scratch
+    (1, 8, 4096, 256, 128, 8, 2),
+]
+
+
+@pytest.mark.parametrize("case", CASES)
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
-def test_noalloc_matches_workspace_entry_point(lib, out_dtype):
-    B, H, Sq, Skv, D, n_split = 1, 8, 300, 5000, 128, 4
+def test_noalloc_matches_workspace_entry_point(lib, case, out_dtype):
+    B, H, Sq, Skv, D, n_split, n_used = case
     dt = BF16 if out_dtype == torch.bfloat16 else F32
-    g = torch.Generator().manual_seed(123)
+    g = torch.Generator().manual_seed(123 + Sq)
     q, k, v = (torch.randn(B, s, H, D, generator=g).to(torch.bfloat16).cuda()
                for s in (Sq, Skv, Skv))
     k2, v2 = (torch.randn(B, Skv, H, D, generator=g).to(torch.bfloat16).cuda() for _ in range(2))
     scale = 1.0 / math.sqrt(D)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    need = lib.cpattn_fwd_split_workspace(B, H, Sq, D, n_split, dt)
+    need = lib.cpattn_fwd_split_workspace(B, H, Sq, D, n_used, dt)
     assert 0 < need <= lib.cpattn_noalloc_scratch_bytes()
+    if n_used != n_split:  # the unlowered request alone would not fit
+        assert lib.cpattn_fwd_split_workspace(B, H, Sq, D, n_split, dt) > \
+            lib.cpattn_noalloc_scratch_bytes()
     ws = torch.empty(need, dtype=torch.uint8, device="cuda")
 
     o_ref = torch.empty(B, Sq, H, D, dtype=out_dtype, device="cuda")
@@ -73,11 +90,31 @@ def test_noalloc_matches_workspace_entry_point(lib, out_dtype):
                                           Skv, D, scale, dt, acc, n_split, stream)
         assert st == OK, st
         torch.cuda.synchronize()
-        # the same kernels on the same data: within the tolerance the parity tests use
-        # (1e-2 on O, 1e-3 on LSE); in practice identical
-        assert (o_na.float() - o_ref.float()).abs().max().item() <= 1e-2, call
-        assert (l_na - l_ref).abs().max().item() <= 1e-3, call
+        # the same kernels on the same data and the same partial layout: identical bits
+        assert torch.equal(o_na, o_ref), call
+        assert torch.equal(l_na, l_ref), call
         assert torch.isfinite(o_na.float()).all() and torch.isfinite(l_na).all()
+    assert lib.cpattn_device_error() == OK
+
+
+def test_noalloc_call_allocates_nothing(lib):
+    B, H, Sq, Skv, D, n_split = 1, 4, 500, 3000, 128, 4
+    g = torch.Generator().manual_seed(5)
+    q, k, v = (torch.randn(B, s, H, D, generator=g).to(torch.bfloat16).cuda()
+               for s in (Sq, Skv, Skv))
+    o = torch.empty(B, Sq, H, D, dtype=torch.bfloat16, device="cuda")
+    l = torch.empty(B, H, Sq, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    args = (_p(q), _p(k), _p(v), _p(o), _p(l), B, H, Sq, Skv, D, 1.0 / math.sqrt(D), BF16, 0,
+            n_split, stream)
+    assert lib.cpattn_fwd_split_noalloc(*args) == OK  # warm-up: the first call on a device
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        assert lib.cpattn_fwd_split_noalloc(*args) == OK
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, (free0, free1)
     assert lib.cpattn_device_error() == OK
 
 
