@@ -186,19 +186,22 @@ size_t cpattn_fwd_split_workspace(int B, int H, int Sq, int D, int n_split, int 
 
 int cpattn_split_suggest(int B, int H, int Sq, int Skv) {
   if (B < 1 || H < 1 || Sq < 1 || Skv < 1) return 1;
-  const long long ctas = (long long)((Sq + 255) / 256) * H * B;
+  // Work items are (256-row query tile pair, head, key range); the persistent attention
+  // kernel runs them round-robin on one CTA per SM.  Modelled time in units of one key
+  // block of one item (~2 us at the S = 44160 rate): rounds of items that each do 1/s of
+  // the key blocks plus about one block of per-item epilogue, plus, for s > 1, the combine
+  // pass, which streams s partials and the result (bf16, D = 128 assumed) at ~6 TB/s.
+  const long long items = (long long)((Sq + 255) / 256) * H * B;
   const int sms = cpattn::sm_count();
   const int n_kv = (Skv + 127) / 128;
-  if (ctas >= 4LL * sms) return 1;  // already four or more waves: little tail to recover
-  // modelled time per split count: waves of CTAs that each do 1/s of the key blocks, plus
-  // a per-CTA start-up (prologue, pipeline fill, epilogue) worth ~10 key blocks -- measured:
-  // a 352-CTA grid of 43-block CTAs gains nothing from two ranges -- and a combine pass of
-  // ~1 block per split
+  const double out_bytes = double(B) * Sq * H * 128 * 2;
+  const double block_us = 2.1, hbm_bytes_per_us = 6.0e6;
   double best = 1e30;
   int best_s = 1;
   for (int sp = 1; sp <= kMaxSplit && n_kv / sp >= 4; ++sp) {
-    const long long waves = (ctas * sp + sms - 1) / sms;
-    const double t = double(waves) * (double(n_kv) / sp + 10.0) + (sp > 1 ? sp : 0);
+    const long long rounds = (items * sp + sms - 1) / sms;
+    double t = double(rounds) * (double(n_kv) / sp + 1.0);
+    if (sp > 1) t += (sp + 2) * out_bytes / hbm_bytes_per_us / block_us;
     if (t < best * 0.97) {
       best = t;
       best_s = sp;

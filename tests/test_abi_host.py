@@ -123,9 +123,13 @@ def test_fwd_split_argument_errors_and_sizes(L):
 
 
 def test_split_suggestion_model():
-    assert B.split_suggest(8, 2, 44160, 44160) == 1  # 2768 CTAs: many waves already
-    assert B.split_suggest(1, 16, 512, 44160) >= 4   # 32 CTAs over 345 key blocks: split
-    assert B.split_suggest(1, 16, 5520, 5520) == 1   # 352 CTAs of 43 blocks: start-up eats it
+    # work items are (256-row tile pair, head, key range) on 148 persistent CTAs (no GPU
+    # here: the library's default SM count)
+    assert B.split_suggest(8, 2, 44160, 44160) == 1  # 2768 items: 18.7 rounds already
+    assert B.split_suggest(1, 24, 4608, 4608) == 1   # 432 items: 2.92 rounds, nothing to gain
+    assert B.split_suggest(1, 16, 512, 44160) == 4   # 32 items over 345 key blocks: split
+    # 352 items of 43 blocks = 2.38 rounds; two ranges give 704 half items = 4.76 rounds
+    assert B.split_suggest(1, 16, 5520, 5520) == 2
     assert B.split_suggest(1, 1, 128, 128) == 1       # too few key blocks to split
 
 

@@ -187,6 +187,65 @@ def test_bf16_shapes_match_oracle(shape):
     assert rel_l2(o32, o_ref) < 1e-2
 
 
+# The attention kernel is persistent: at most one CTA per SM (148 on B200) loops over work
+# items of (256-row query tile pair, head, batch).  These shapes give CTAs several items
+# each, with ragged query and key tails, single-block items and both head widths, so that
+# the pipeline's hand-over from one item to the next (Q reload, O read-out while the next
+# item's S is computed) is checked element by element.
+MULTI_ITEM_SHAPES = [(2, 40, 300, 257, 128), (1, 96, 600, 130, 64), (1, 150, 256, 100, 128),
+                     (3, 70, 513, 384, 128)]
+
+
+@pytest.mark.parametrize("shape", MULTI_ITEM_SHAPES)
+def test_persistent_items_match_oracle(shape):
+    Bn, H, Sq, Skv, D = shape
+    q, k, v = W.random_case(7 * Sq + H, Bn, H, Sq, Skv, D)
+    scale = 1.0 / math.sqrt(D)
+    o_ref, l_ref = ref.attention(q, k, v, scale)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    o32, l32 = cp.fwd(qd, kd, vd, scale=scale, out_dtype=torch.float32)
+    o16, l16 = cp.fwd(qd, kd, vd, scale=scale)
+    torch.cuda.synchronize()
+    check_o(o32, o_ref, "bf16_in", f"{shape} fp32 epilogue")
+    check_o(o16, o_ref, "bf16_out", f"{shape} bf16 out")
+    check_lse(l32, l_ref, str(shape))
+    assert torch.equal(l16, l32)
+    assert rel_l2(o32, o_ref) < 1e-2
+    # the same items as a two-chunk ring step (accumulate) and as split-KV ranges
+    c = Skv // 2
+    o_acc = torch.full((Bn, Sq, H, D), float("nan"), dtype=torch.float32, device=DEV)
+    l_acc = torch.full((Bn, H, Sq), -math.inf, device=DEV)
+    for a, b in ((0, c), (c, Skv)):
+        cp.fwd_accumulate(qd, kd[:, a:b].contiguous(), vd[:, a:b].contiguous(), o_acc, l_acc,
+                          scale=scale)
+    o_s, l_s = cp.fwd_split(qd, kd, vd, out_dtype=torch.float32, n_split=3)
+    torch.cuda.synchronize()
+    check_o(o_acc, o_ref, "bf16_in", f"{shape} ring of 2")
+    check_lse(l_acc, l_ref, f"{shape} ring of 2")
+    check_o(o_s, o_ref, "bf16_in", f"{shape} split 3")
+    check_lse(l_s, l_ref, f"{shape} split 3")
+
+
+def test_persistent_fused_ulysses_many_items():
+    # 4 ranks x 400 tokens, 64 heads: 7 tile pairs x 16 heads x 4 groups = 448 items
+    P, S_l, H, D = 4, 400, 64, 128
+    g = torch.Generator().manual_seed(404)
+    shards = [W.randn((P, S_l, H, D), g, 1.0, "bf16").to(DEV) for _ in range(3)]
+    out_f, lse_f = cp.ulysses_fwd(*shards, P, out_dtype=torch.float32)
+    qh, kh, vh = (cp.seq2head(t, P) for t in shards)
+    oh, lse_u = cp.fwd(qh, kh, vh, out_dtype=torch.float32)
+    out_u = cp.head2seq(oh, P)
+    torch.cuda.synchronize()
+    assert torch.equal(out_f, out_u) and torch.equal(lse_f, lse_u)
+    full = lambda t: t.cpu().reshape(1, P * S_l, H, D)
+    rows = W.sample_rows(1, H, P * S_l, 1024, seed=8)
+    o_ref, l_ref = ref.attention_rows(full(shards[0]), full(shards[1]), full(shards[2]),
+                                      1 / math.sqrt(D), rows)
+    oc, lc = out_f.cpu().reshape(1, P * S_l, H, D), lse_f.cpu().reshape(1, H, P * S_l)
+    check_o(torch.stack([oc[b, i, h] for (b, h, i) in rows]), o_ref, "bf16_in", "ulysses items")
+    check_lse(torch.stack([lc[b, h, i] for (b, h, i) in rows]), l_ref, "ulysses items")
+
+
 @pytest.mark.parametrize("shape,split", [((1, 2, 130, 300, 128), 170), ((2, 1, 257, 129, 64), 1),
                                          ((1, 3, 17, 513, 128), 384)])
 @pytest.mark.parametrize("acc", [torch.bfloat16, torch.float32])
