@@ -530,6 +530,8 @@ def next_paths(cp, w, q, k, v, plan, dev, stream):
     ms_u = timed(lambda: cp.ring_attention(q3, kc, vc, scale=w3.softmax_scale, fused=False))
     ms_s = timed(lambda: cp.ring_attention(q3, kc, vc, scale=w3.softmax_scale, fused=True,
                                            n_split=n_split))
+    ms_t = timed(lambda: cp.ring_attention(q3, kc, vc, scale=w3.softmax_scale, fused=True,
+                                           n_split=0))
     # AllGather-KV-like: a short query slice (512 tokens, 16 heads) against all 44160 keys --
     # 32 CTAs for 148 SMs, the case split-KV is for
     g = torch.Generator(device="cpu").manual_seed(41)
@@ -552,29 +554,57 @@ def next_paths(cp, w, q, k, v, plan, dev, stream):
         "unfused_ms": round(ms_u, 4), "unfused_TFLOP/s": round(w3.attn_flops / ms_u / 1e9, 2),
         "split_kv": n_split, "split_ms": round(ms_s, 4),
         "split_TFLOP/s": round(w3.attn_flops / ms_s / 1e9, 2),
-        "launches_fused": 8, "launches_unfused": 15, "launches_split": 16}
+        "tail_split_ms": round(ms_t, 4), "tail_split_TFLOP/s": round(w3.attn_flops / ms_t / 1e9, 2),
+        "tail_split_frac_of_burst": round(w3.attn_flops / ms_t / 1e9 / peaks["bf16_tflops"], 4),
+        "tail_split": ("352 items on 148 SMs: 296 whole, the 56 of the last wave as 2 key "
+                       "ranges each, folded into the accumulator by a combine kernel"),
+        "launches_fused": 8, "launches_unfused": 15, "launches_split": 16,
+        "launches_tail_split": 16}
     return res
 
 
 def e2e_run(cp, UlyssesPlan, w, x, dev, stream, args):
-    """Same metric through the public API with pinned host buffers: every step copies its
-    Q/K/V shards host -> device and its O and LSE device -> host inside the timed region.
+    """Same metric end to end with pinned host buffers: every step copies its Q/K/V shards
+    host -> device and its O and LSE device -> host inside the timed region.
 
-    ``pipelined`` (the reported value): ``UlyssesStreamer`` overlaps the copies of
-    neighbouring steps with compute (two device buffer sets, upload/compute/download
-    streams), as a serving loop would run; timed from the first upload to the last
-    download.  ``serial``: copy in, compute, copy out, one step after another."""
-    from context_long_sequence_non_b200.paths import UlyssesStreamer
+    The reported value goes through the C ABI's host-buffer call (cpattn_ulysses_host via
+    ``UlyssesHostPass``): inside each call the head groups go in chunks, and the upload of
+    one chunk and the download of another overlap the attention of a third.  Calls run
+    back to back on one stream, each ordered after the previous one.  Also reported:
+    ``streamer`` (``UlyssesStreamer``: whole steps overlapped with their neighbours' copies
+    on three streams, as a serving loop would run them) and ``serial`` (copy in, compute,
+    copy out, one step after another)."""
+    from context_long_sequence_non_b200.paths import UlyssesHostPass, UlyssesStreamer
 
     P, S_l, H = w.P, w.Sq // w.P, w.H * w.P
     hq, hk, hv = (x[n].pin_memory() for n in ("q", "k", "v"))
     plan = UlyssesPlan(P, S_l, H, w.D, device=dev)
-    dq, dk, dv = (torch.empty_like(hq, device=dev) for _ in range(3))
     ho = torch.empty(plan.out.shape, dtype=plan.out.dtype).pin_memory()
     hl = torch.empty(plan.lse.shape, dtype=plan.lse.dtype).pin_memory()
     n = max(3, min(args.steps, 10))
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+
+    def timed(fn, start_stream=None, end_stream=None):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(start_stream or stream)
+        for _ in range(n):
+            fn()
+        b.record(end_stream or stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / n
+
+    tf = lambda ms: round(w.attn_flops / (ms * 1e-3) / 1e12, 2)
+
+    # through the C ABI: host shards in, host O/LSE out, copies pipelined inside the call
+    hp = UlyssesHostPass(P, S_l, H, w.D, device=dev)
+    ms_host = timed(lambda: hp.run(hq, hk, hv, ho, hl, scale=w.softmax_scale))
+    del hp
+
+    dq, dk, dv = (torch.empty_like(hq, device=dev) for _ in range(3))
 
     def serial_step():
         dq.copy_(hq, non_blocking=True)
@@ -584,38 +614,29 @@ def e2e_run(cp, UlyssesPlan, w, x, dev, stream, args):
         ho.copy_(plan.out, non_blocking=True)
         hl.copy_(plan.lse, non_blocking=True)
 
-    for _ in range(2):
-        serial_step()
-    torch.cuda.synchronize(dev)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(n):
-        serial_step()
-    b.record(stream)
-    torch.cuda.synchronize(dev)
-    ms_serial = a.elapsed_time(b) / n
+    ms_serial = timed(serial_step)
     del plan, dq, dk, dv
 
-    # pipelined: two host output sets so a step's download never races the next step's
+    # whole steps overlapped: two host output sets so a step's download never races the next
     streamer = UlyssesStreamer(P, S_l, H, w.D, device=dev, depth=2)
     outs = [(ho, hl), (torch.empty_like(ho).pin_memory(), torch.empty_like(hl).pin_memory())]
-    for i in range(2):
-        streamer.submit(hq, hk, hv, *outs[i % 2], scale=w.softmax_scale)
-    torch.cuda.synchronize(dev)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(streamer.upload)
-    for i in range(n):
-        streamer.submit(hq, hk, hv, *outs[i % 2], scale=w.softmax_scale)
-    b.record(streamer.download)
-    torch.cuda.synchronize(dev)
-    ms = a.elapsed_time(b) / n
-    return {"value": round(w.attn_flops / (ms * 1e-3) / 1e12, 2), "unit": UNIT,
-            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "steps": n, "mode": "pipelined: UlyssesStreamer, copies of neighbouring steps "
-                                "overlap compute (2 buffer sets, upload/compute/download streams)",
-            "serial": {"value": round(w.attn_flops / (ms_serial * 1e-3) / 1e12, 2),
-                       "ms_per_step": round(ms_serial, 4),
-                       "mode": "copy in, compute, copy out, one step after another"}}
+    k = [0]
+
+    def stream_step():
+        streamer.submit(hq, hk, hv, *outs[k[0] % 2], scale=w.softmax_scale)
+        k[0] += 1
+
+    ms_streamer = timed(stream_step, streamer.upload, streamer.download)
+    return {"value": tf(ms_host), "unit": UNIT, "ms_per_step": round(ms_host, 4),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
+            "mode": ("C ABI cpattn_ulysses_host (UlyssesHostPass): pinned host Q/K/V shards in, "
+                     "host O + LSE out; head groups in 4 chunks, uploads and downloads "
+                     "overlapping the attention inside each call; calls back to back"),
+            "streamer": {"value": tf(ms_streamer), "ms_per_step": round(ms_streamer, 4),
+                         "mode": "UlyssesStreamer: neighbouring steps' copies overlap compute "
+                                 "(2 buffer sets, upload/compute/download streams)"},
+            "serial": {"value": tf(ms_serial), "ms_per_step": round(ms_serial, 4),
+                       "mode": "copy in, compute (5 launches), copy out, one step after another"}}
 
 
 # --------------------------------------------------------------------------- CPU oracle

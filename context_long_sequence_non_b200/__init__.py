@@ -5,6 +5,8 @@
 * ``seq2head``  Ulysses sequence shards -> head groups over P virtual ranks
 * ``head2seq``  the inverse permute
 * ``ring_attention`` / ``ulysses_attention``  the two per-rank compositions
+* ``UlyssesHostPass``  a whole Ulysses layer from host shards to host O/LSE, copies
+  pipelined with the attention inside the library (cpattn_ulysses_host)
 
 All compute runs in ``libcpattn.so`` (C ABI in ``include/cpattn.h``); this package only
 marshals arguments.  ``workloads`` holds the seeded synthetic inputs.
@@ -21,6 +23,7 @@ from ._binding import (  # noqa: F401
     split_suggest,
     split_workspace_bytes,
     ulysses_fwd,
+    ulysses_host,
     head2seq,
     lib,
     library_path,
@@ -34,4 +37,10 @@ from ._binding import (  # noqa: F401
     status_str,
     version,
 )
-from .paths import UlyssesPlan, UlyssesStreamer, ring_attention, ulysses_attention  # noqa: F401
+from .paths import (  # noqa: F401
+    UlyssesHostPass,
+    UlyssesPlan,
+    UlyssesStreamer,
+    ring_attention,
+    ulysses_attention,
+)

@@ -49,6 +49,8 @@ def lib() -> ctypes.CDLL:
             L.cpattn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
             L.cpattn_fwd_accumulate.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
             L.cpattn_ulysses_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+            L.cpattn_ulysses_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i,
+                                              f, i, i, vp]
             L.cpattn_fwd_split.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp,
                                            ctypes.c_size_t, vp]
             L.cpattn_fwd_split_workspace.argtypes = [i, i, i, i, i, i]
@@ -68,6 +70,7 @@ def lib() -> ctypes.CDLL:
             L.cpattn_version.argtypes = []
             L.cpattn_selftest_exp2.argtypes = [vp, vp, i, vp]
             for name in ("cpattn_fwd", "cpattn_fwd_accumulate", "cpattn_ulysses_fwd",
+                         "cpattn_ulysses_host",
                          "cpattn_fwd_split", "cpattn_split_suggest", "cpattn_merge", "cpattn_seq2head_qkv", "cpattn_seq2head", "cpattn_head2seq",
                          "cpattn_device_error", "cpattn_selftest_wait_timeout", "cpattn_version",
                          "cpattn_selftest_exp2"):
@@ -156,6 +159,36 @@ def ulysses_fwd(q, k, v, P, out=None, lse=None, scale=None, out_dtype=None, want
                                   float(scale), _dtype_code(out.dtype), _stream(stream))
     _check(st, "cpattn_ulysses_fwd")
     return out, lse
+
+
+def ulysses_host(hq, hk, hv, h_out, h_lse, dq, dk, dv, d_out, d_lse, P, scale=None,
+                 n_chunks=None, stream=None):
+    """Ulysses attention from host shards to host O/LSE through cpattn_ulysses_host: the
+    copies are pipelined with the attention over head-group chunks.  h_*: CPU tensors
+    (pinned for asynchronous copies); d_*: same-shaped CUDA work buffers.  The host
+    outputs are valid once ``stream`` (default: the current stream) has passed the call."""
+    P_, S_l, H, D = hq.shape
+    for t in (hk, hv, dq, dk, dv):
+        if t.shape != hq.shape:
+            raise ValueError("all shard tensors must be [P][S_l][H][D]")
+    if h_out.shape != hq.shape or d_out.shape != hq.shape or h_out.dtype != d_out.dtype:
+        raise ValueError("h_out and d_out must be [P][S_l][H][D] of one dtype")
+    if (h_lse is None) != (d_lse is None):
+        raise ValueError("h_lse and d_lse go together")
+    for t in (hq, hk, hv, h_out, h_lse):
+        if t is not None and (t.is_cuda or not t.is_contiguous()):
+            raise ValueError("host tensors must be contiguous CPU tensors")
+    _need_cuda(dq, dk, dv, d_out, d_lse)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if n_chunks is None:
+        n_chunks = max(1, P // 2)
+    st = lib().cpattn_ulysses_host(_ptr(hq), _ptr(hk), _ptr(hv), _ptr(h_out), _ptr(h_lse),
+                                   _ptr(dq), _ptr(dk), _ptr(dv), _ptr(d_out), _ptr(d_lse), P,
+                                   S_l, H, D, float(scale), _dtype_code(d_out.dtype),
+                                   int(n_chunks), _stream(stream))
+    _check(st, "cpattn_ulysses_host")
+    return h_out, h_lse
 
 
 def split_workspace_bytes(B, H, Sq, D, n_split, out_dtype=torch.bfloat16) -> int:

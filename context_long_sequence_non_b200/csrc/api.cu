@@ -179,29 +179,32 @@ extern "C" {
 
 size_t cpattn_fwd_split_workspace(int B, int H, int Sq, int D, int n_split, int out_dtype) {
   const int es = elem_size(out_dtype);
-  if (B < 1 || H < 1 || Sq < 1 || D < 1 || n_split < 1 || n_split > kMaxSplit || es == 0)
+  if (B < 1 || H < 1 || Sq < 1 || D < 1 || n_split < 0 || n_split > kMaxSplit || es == 0)
     return 0;
+  if (n_split == 0) {
+    // tail split: the plan depends on the key count only through "at least 2 blocks per
+    // range"; size the workspace for the most parts any key count can give
+    if (D != 64 && D != 128) return 0;
+    return cpattn::tail_split_workspace(cpattn::tail_split_plan(B, H, Sq, 1 << 30), D);
+  }
   return n_split == 1 ? 0 : split_ws_bytes(B, H, Sq, D, n_split, es);
 }
 
 int cpattn_split_suggest(int B, int H, int Sq, int Skv) {
   if (B < 1 || H < 1 || Sq < 1 || Skv < 1) return 1;
-  // Work items are (256-row query tile pair, head, key range); the persistent attention
-  // kernel runs them round-robin on one CTA per SM.  Modelled time in units of one key
-  // block of one item (~2 us at the S = 44160 rate): rounds of items that each do 1/s of
-  // the key blocks plus about one block of per-item epilogue, plus, for s > 1, the combine
-  // pass, which streams s partials and the result (bf16, D = 128 assumed) at ~6 TB/s.
-  const long long items = (long long)((Sq + 255) / 256) * H * B;
+  const long long ctas = (long long)((Sq + 255) / 256) * H * B;
   const int sms = cpattn::sm_count();
   const int n_kv = (Skv + 127) / 128;
-  const double out_bytes = double(B) * Sq * H * 128 * 2;
-  const double block_us = 2.1, hbm_bytes_per_us = 6.0e6;
+  if (ctas >= 4LL * sms) return 1;  // already four or more waves: little tail to recover
+  // modelled time per split count: waves of CTAs that each do 1/s of the key blocks, plus
+  // a per-CTA start-up (prologue, pipeline fill, epilogue) worth ~10 key blocks -- measured:
+  // a 352-CTA grid of 43-block CTAs gains nothing from two ranges -- and a combine pass of
+  // ~1 block per split
   double best = 1e30;
   int best_s = 1;
   for (int sp = 1; sp <= kMaxSplit && n_kv / sp >= 4; ++sp) {
-    const long long rounds = (items * sp + sms - 1) / sms;
-    double t = double(rounds) * (double(n_kv) / sp + 1.0);
-    if (sp > 1) t += (sp + 2) * out_bytes / hbm_bytes_per_us / block_us;
+    const long long waves = (ctas * sp + sms - 1) / sms;
+    const double t = double(waves) * (double(n_kv) / sp + 10.0) + (sp > 1 ? sp : 0);
     if (t < best * 0.97) {
       best = t;
       best_s = sp;
@@ -214,9 +217,15 @@ int cpattn_fwd_split(const void* q, const void* k, const void* v, void* out, flo
                      int H, int Sq, int Skv, int D, float scale, int out_dtype, int accumulate,
                      int n_split, void* workspace, size_t workspace_bytes,
                      cpattn_stream_t stream) {
-  if (n_split < 1 || n_split > kMaxSplit) return CPATTN_ERR_SHAPE;
+  if (n_split < 0 || n_split > kMaxSplit) return CPATTN_ERR_SHAPE;
   const int n_kv = Skv > 0 ? (Skv + 127) / 128 : 0;
-  if (n_split > n_kv) n_split = n_kv > 0 ? n_kv : 1;  // every range holds a key block
+  cpattn::TailSplit tail{};
+  if (n_split == 0) {  // tail split: only the items of the last, partial wave are split
+    if (B >= 1 && H >= 1 && Sq >= 1 && Skv >= 1) tail = cpattn::tail_split_plan(B, H, Sq, Skv);
+    if (tail.parts < 2) n_split = 1;
+  } else if (n_split > n_kv) {
+    n_split = n_kv > 0 ? n_kv : 1;  // every range holds a key block
+  }
   if (n_split == 1)
     return fwd_impl(q, k, v, out, lse, B, H, Sq, Skv, D, scale, CPATTN_BF16, out_dtype,
                     accumulate != 0, stream);
@@ -232,7 +241,9 @@ int cpattn_fwd_split(const void* q, const void* k, const void* v, void* out, flo
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
       !aligned(workspace, 256) || (lse != nullptr && !aligned(lse, 4)))
     return CPATTN_ERR_ALIGN;
-  if (workspace_bytes < split_ws_bytes(B, H, Sq, D, n_split, es)) return CPATTN_ERR_SHAPE;
+  const size_t need = n_split == 0 ? cpattn::tail_split_workspace(tail, D)
+                                    : split_ws_bytes(B, H, Sq, D, n_split, es);
+  if (workspace_bytes < need) return CPATTN_ERR_SHAPE;
   if ((long long)B * Sq * H > 0x7fffffffLL) return CPATTN_ERR_SHAPE;  // 32-bit row index
   int* err = device_error_word();
   if (err == nullptr) return CPATTN_ERR_CUDA;
@@ -241,6 +252,13 @@ int cpattn_fwd_split(const void* q, const void* k, const void* v, void* out, flo
       !encode_bshd_bf16(&tv, v, B, Skv, H, D))
     return CPATTN_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (n_split == 0) {
+    const float scale_log2 = float(double(scale) * 1.4426950408889634074);
+    return cuda_status(cpattn::launch_attn_fwd_sm100_tail(
+        tq, tk, tv, out, lse, B, H, Sq, Skv, D, scale_log2, cpattn::kRescaleLog2,
+        out_dtype == CPATTN_F32, accumulate != 0, tail, workspace, err, cpattn::kDefaultWaitLimit,
+        st));
+  }
   void* part_o = workspace;
   float* part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                              split_o_bytes(B, H, Sq, D, n_split, es));
@@ -253,9 +271,13 @@ int cpattn_fwd_split(const void* q, const void* k, const void* v, void* out, flo
                                             accumulate != 0, st));
 }
 
-int cpattn_ulysses_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int P,
-                       int S_local, int H, int D, float scale, int out_dtype,
-                       cpattn_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Checks shared by the device and host Ulysses calls (no CUDA call).
+int ulysses_args(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                 int P, int S_local, int H, int D, float scale, int out_dtype) {
   if (P < 1 || S_local < 1 || H < 1 || D < 1) return CPATTN_ERR_SHAPE;
   if (H % P != 0) return CPATTN_ERR_SHAPE;
   if ((long long)P * S_local > 0x7fffffffLL || P > 65535 || H / P > 65535) return CPATTN_ERR_SHAPE;
@@ -267,20 +289,154 @@ int cpattn_ulysses_fwd(const void* q, const void* k, const void* v, void* out, f
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
       (lse != nullptr && !aligned(lse, 4)))
     return CPATTN_ERR_ALIGN;
+  return CPATTN_OK;
+}
+
+struct UlyssesMaps {
+  CUtensorMap q, k, v, q16, k16, v16;
+};
+
+bool encode_ulysses(UlyssesMaps* m, const void* q, const void* k, const void* v, int P,
+                    int S_local, int H, int D) {
+  return encode_bshd_bf16(&m->q, q, P, S_local, H, D) && encode_bshd_bf16(&m->k, k, P, S_local, H, D) &&
+         encode_bshd_bf16(&m->v, v, P, S_local, H, D) &&
+         encode_bshd_bf16(&m->q16, q, P, S_local, H, D, 16) &&
+         encode_bshd_bf16(&m->k16, k, P, S_local, H, D, 16) &&
+         encode_bshd_bf16(&m->v16, v, P, S_local, H, D, 16);
+}
+
+// Per-device streams and events of the host-buffer pass, created on the first call on a
+// device and kept until the process exits (no device memory is involved).  The mutex is
+// held while a call enqueues its work, so that one event can be recorded and waited on
+// again and again: every wait is enqueued right after the record it refers to.
+struct HostPassResources {
+  std::mutex mu;
+  bool ready = false;
+  cudaStream_t upload = nullptr, download = nullptr, compute2 = nullptr;
+  cudaEvent_t start = nullptr, uploaded = nullptr, computed = nullptr, done = nullptr;
+};
+
+HostPassResources* host_pass_resources(int* status) {
+  static HostPassResources res[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    *status = CPATTN_ERR_CUDA;
+    return nullptr;
+  }
+  HostPassResources* r = &res[dev];
+  *status = CPATTN_OK;
+  return r;
+}
+
+bool host_pass_init(HostPassResources* r) {  // with r->mu held
+  if (r->ready) return true;
+  const unsigned sf = cudaStreamNonBlocking, ef = cudaEventDisableTiming;
+  if (cudaStreamCreateWithFlags(&r->upload, sf) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&r->download, sf) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&r->compute2, sf) != cudaSuccess ||
+      cudaEventCreateWithFlags(&r->start, ef) != cudaSuccess ||
+      cudaEventCreateWithFlags(&r->uploaded, ef) != cudaSuccess ||
+      cudaEventCreateWithFlags(&r->computed, ef) != cudaSuccess ||
+      cudaEventCreateWithFlags(&r->done, ef) != cudaSuccess)
+    return false;
+  r->ready = true;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+int cpattn_ulysses_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int P,
+                       int S_local, int H, int D, float scale, int out_dtype,
+                       cpattn_stream_t stream) {
+  const int st = ulysses_args(q, k, v, out, lse, P, S_local, H, D, scale, out_dtype);
+  if (st != CPATTN_OK) return st;
   int* err = device_error_word();
   if (err == nullptr) return CPATTN_ERR_CUDA;
-  CUtensorMap tq, tk, tv, tq16, tk16, tv16;
-  if (!encode_bshd_bf16(&tq, q, P, S_local, H, D) || !encode_bshd_bf16(&tk, k, P, S_local, H, D) ||
-      !encode_bshd_bf16(&tv, v, P, S_local, H, D) ||
-      !encode_bshd_bf16(&tq16, q, P, S_local, H, D, 16) ||
-      !encode_bshd_bf16(&tk16, k, P, S_local, H, D, 16) ||
-      !encode_bshd_bf16(&tv16, v, P, S_local, H, D, 16))
-    return CPATTN_ERR_CUDA;
+  UlyssesMaps m;
+  if (!encode_ulysses(&m, q, k, v, P, S_local, H, D)) return CPATTN_ERR_CUDA;
   const float scale_log2 = float(double(scale) * 1.4426950408889634074);
   return cuda_status(cpattn::launch_ulysses_fwd_sm100(
-      tq, tk, tv, tq16, tk16, tv16, out, lse, P, S_local, H, D, scale_log2, cpattn::kRescaleLog2,
-      out_dtype == CPATTN_F32, err, cpattn::kDefaultWaitLimit,
+      m.q, m.k, m.v, m.q16, m.k16, m.v16, out, lse, P, S_local, H, D, scale_log2,
+      cpattn::kRescaleLog2, out_dtype == CPATTN_F32, 0, P, err, cpattn::kDefaultWaitLimit,
       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int cpattn_ulysses_host(const void* h_q, const void* h_k, const void* h_v, void* h_out,
+                        float* h_lse, void* d_q, void* d_k, void* d_v, void* d_out, float* d_lse,
+                        int P, int S_local, int H, int D, float scale, int out_dtype, int n_chunks,
+                        cpattn_stream_t stream) {
+  const int st = ulysses_args(d_q, d_k, d_v, d_out, d_lse, P, S_local, H, D, scale, out_dtype);
+  if (st != CPATTN_OK) return st;
+  if (n_chunks < 1 || n_chunks > P) return CPATTN_ERR_SHAPE;
+  if (!h_q || !h_k || !h_v || !h_out) return CPATTN_ERR_NULL;
+  if ((h_lse == nullptr) != (d_lse == nullptr)) return CPATTN_ERR_NULL;
+  const int es = elem_size(out_dtype);
+  const size_t in_bytes = size_t(P) * S_local * H * D * 2, out_bytes = in_bytes / 2 * es;
+  const size_t lse_bytes = size_t(H) * P * S_local * 4;
+  const void* dev_bufs[5] = {d_q, d_k, d_v, d_out, d_lse};
+  const size_t dev_sizes[5] = {in_bytes, in_bytes, in_bytes, out_bytes, lse_bytes};
+  for (int a = 0; a < 5; ++a)
+    for (int b = a + 1; b < 5; ++b)
+      if (dev_bufs[a] && dev_bufs[b] && overlap(dev_bufs[a], dev_sizes[a], dev_bufs[b], dev_sizes[b]))
+        return CPATTN_ERR_SHAPE;
+  int* err = device_error_word();
+  if (err == nullptr) return CPATTN_ERR_CUDA;
+  UlyssesMaps m;
+  if (!encode_ulysses(&m, d_q, d_k, d_v, P, S_local, H, D)) return CPATTN_ERR_CUDA;
+  int rs = CPATTN_OK;
+  HostPassResources* r = host_pass_resources(&rs);
+  if (r == nullptr) return rs;
+  std::lock_guard<std::mutex> lock(r->mu);
+  if (!host_pass_init(r)) return CPATTN_ERR_CUDA;
+  cudaStream_t cs[2] = {reinterpret_cast<cudaStream_t>(stream), r->compute2};
+  const float scale_log2 = float(double(scale) * 1.4426950408889634074);
+  const int Hp = H / P;
+  const size_t rows = size_t(P) * S_local;  // token rows of every shard tensor
+  // everything below is ordered after the work already on the caller's stream
+  cudaError_t e = cudaEventRecord(r->start, cs[0]);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(r->upload, r->start, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(r->download, r->start, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(cs[1], r->start, 0);
+  for (int c = 0; e == cudaSuccess && c < n_chunks; ++c) {
+    // chunk c = head groups [g0, g1): heads [g0*Hp, g1*Hp) of every token row, a strided
+    // slab of each [P][S_l][H][D] tensor (one 2-D copy per tensor and direction)
+    const int g0 = int((long long)c * P / n_chunks), g1 = int((long long)(c + 1) * P / n_chunks);
+    const size_t in_off = size_t(g0) * Hp * D * 2, in_w = size_t(g1 - g0) * Hp * D * 2;
+    const size_t in_pitch = size_t(H) * D * 2;
+    const void* hs[3] = {h_q, h_k, h_v};
+    void* ds[3] = {d_q, d_k, d_v};
+    for (int t = 0; e == cudaSuccess && t < 3; ++t)
+      e = cudaMemcpy2DAsync(static_cast<char*>(ds[t]) + in_off, in_pitch,
+                            static_cast<const char*>(hs[t]) + in_off, in_pitch, in_w, rows,
+                            cudaMemcpyHostToDevice, r->upload);
+    if (e == cudaSuccess) e = cudaEventRecord(r->uploaded, r->upload);
+    cudaStream_t s = cs[c & 1];  // neighbouring chunks overlap on two compute streams
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, r->uploaded, 0);
+    if (e == cudaSuccess)
+      e = cpattn::launch_ulysses_fwd_sm100(m.q, m.k, m.v, m.q16, m.k16, m.v16, d_out, d_lse, P,
+                                           S_local, H, D, scale_log2, cpattn::kRescaleLog2,
+                                           out_dtype == CPATTN_F32, g0, g1 - g0, err,
+                                           cpattn::kDefaultWaitLimit, s);
+    if (e == cudaSuccess) e = cudaEventRecord(r->computed, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(r->download, r->computed, 0);
+    const size_t out_off = size_t(g0) * Hp * D * es, out_w = size_t(g1 - g0) * Hp * D * es;
+    const size_t out_pitch = size_t(H) * D * es;
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(static_cast<char*>(h_out) + out_off, out_pitch,
+                            static_cast<const char*>(d_out) + out_off, out_pitch, out_w, rows,
+                            cudaMemcpyDeviceToHost, r->download);
+    if (e == cudaSuccess && h_lse != nullptr) {
+      const size_t l_off = size_t(g0) * Hp * rows, l_n = size_t(g1 - g0) * Hp * rows;
+      e = cudaMemcpyAsync(h_lse + l_off, d_lse + l_off, l_n * 4, cudaMemcpyDeviceToHost,
+                          r->download);
+    }
+  }
+  // the caller's stream resumes once the last copy to the host is done
+  if (e == cudaSuccess) e = cudaEventRecord(r->done, r->download);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(cs[0], r->done, 0);
+  return cuda_status(e);
 }
 
 int cpattn_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b, void* o,

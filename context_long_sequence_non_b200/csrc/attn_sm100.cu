@@ -7,20 +7,21 @@
 // streamed over 128-key blocks with an online softmax, so that the (O, LSE) of separate
 // key chunks merge exactly afterwards (the Ring Attention step).
 //
-// Design: a persistent kernel, one CTA per SM (12 warps), looping over work items.  An
-// item is 256 query rows (two 128-row Q tiles) of one (b, h) against one key range (all
-// keys, or one split-KV range); items are numbered tile-pair fastest, then key range, head,
-// batch, and CTA c takes items c, c + G, c + 2G, ... (G CTAs), so the CTAs running at any
-// moment work on neighbouring items that share their K/V tiles in L2.  Per CTA:
+// Work decomposition.  A work item is 256 query rows (two 128-row Q tiles) of one (b, h)
+// against a range of key blocks.  Two grid forms:
+//   3-D grid (pairs * n_split, H, B): every item over all keys (n_split = 1), or over one of
+//     n_split equal key ranges (split-KV, each range's partial written to its own slice);
+//   1-D grid of n_full + n_tail * tail_parts CTAs ("tail split"): the first n_full items --
+//     whole waves of the GPU -- over all keys, then the n_tail items of the last, partial
+//     wave each split into tail_parts key ranges, so that the last wave is short instead
+//     of mostly idle.  A tail part writes its normalised partial (O, LSE) in fp32 to a
+//     workspace slot; a combine kernel folds the parts (and the running accumulator) after.
+//
+// Design (one CTA = 256 query rows of one (b, h), 12 warps):
 //   warps 0-3  softmax for Q tile 0  (TMEM lanes 0..127, one thread per query row)
 //   warps 4-7  softmax for Q tile 1
-//   warp  8    TMA producer: per item Q0, Q1, then K_0, V_0, K_1, V_1, ... into a 4-slot
-//              ring that runs on across items
+//   warp  8    TMA producer: Q0, Q1 once, then K_0, V_0, K_1, V_1, ... into a 4-slot ring
 //   warp  9    TMEM allocator + single-thread tcgen05.mma issuer
-// Across an item boundary nothing drains: the producer loads the next item's Q as soon as
-// the last Q K^T of the current one has read it, and the issuer computes the next item's
-// first S while the softmax warps write the current item's O; only the next item's first
-// O += P V waits for those warps to have read O out of TMEM.
 // TMEM (512 columns): S0 | S1 (128 fp32 columns each; P_i is written back over S_i as
 // bf16 pairs) | O0 | O1 (D fp32 columns each).  S = Q K^T runs smem x smem; O += P V
 // takes P from TMEM and V from smem (MN-major).  While softmax works on one Q tile the
@@ -46,12 +47,10 @@ constexpr int kSlots = 4;        // K/V ring slots (K_j and V_j alternate)
 constexpr int kThreads = 384;
 constexpr int kWarpProducer = 8;
 constexpr int kWarpMma = 9;
-// Register split (setmaxnreg, multiples of 8): the CTA launches with 168 x 384 = 64512
-// registers; the two softmax warpgroups take 208 each per thread and the producer/MMA
-// warpgroup 88: 2 x 128 x 208 + 128 x 88 = 64512.  The issuer carries the persistent
-// loop's state; at 72 registers it spilled, at 88 (with the Q K^T loop unrolled by 4)
-// nothing spills anywhere.
-constexpr uint32_t kRegsLaunch = 168, kRegsSoftmax = 208, kRegsOther = 88;
+// Register split (setmaxnreg): the CTA launches with 168 x 384 = 64512 registers; the two
+// softmax warpgroups take 216 each per thread and the producer/MMA warpgroup 72:
+// 2 x 128 x 216 + 128 x 72 = 64512 (no spills at this split; 56 spills in the issuer).
+constexpr uint32_t kRegsLaunch = 168, kRegsSoftmax = 216, kRegsOther = 72;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kRegsLaunch * kThreads,
               "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
@@ -81,42 +80,15 @@ struct Geometry {
   static constexpr int kDynSmem = (kBytes + 1024) > 120 * 1024 ? (kBytes + 1024) : 120 * 1024;
 };
 
-// Barrier phases: q_full / q_empty / o_full / o_empty complete once per item, s_full and
-// p_part once per key block (counted over all items of the CTA), full / empty once per use
-// of a ring slot.
 struct __align__(8) Barriers {
-  uint64_t q_full;               // this item's Q0, Q1 landed (TMA transaction count)
-  uint64_t q_empty;              // the item's last Q K^T has read Q (tcgen05.commit)
+  uint64_t q_full;
   uint64_t full[kSlots];
   uint64_t empty[kSlots];
   uint64_t s_full[2];
   uint64_t p_part[2][kPChunks];  // P chunk c of Q tile t stored (chunk 0: O rescaled too)
-  uint64_t o_full[2];            // tile t's last O += P V of the item done
-  uint64_t o_empty[2];           // tile t's softmax warps have read O out of TMEM
+  uint64_t o_full;
   uint64_t drain;
 };
-
-// Work item -> (tile pair, key range, head, batch): tile pair fastest.
-struct Item {
-  int pair, split, h, b;
-};
-__device__ __forceinline__ Item decode_item(int item, int n_pairs, int n_split, int H) {
-  Item it;
-  it.pair = item % n_pairs;
-  int r = item / n_pairs;
-  it.split = r % n_split;
-  r /= n_split;
-  it.h = r % H;
-  it.b = r / H;
-  return it;
-}
-
-// Key blocks [j0, j0 + n) of split range s out of n_split over n_kv_all blocks.
-__device__ __forceinline__ void key_range(int s, int n_split, int n_kv_all, int& j0, int& n) {
-  const int base = n_kv_all / n_split, rem = n_kv_all % n_split;
-  j0 = s * base + (s < rem ? s : rem);
-  n = base + (s < rem ? 1 : 0);
-}
 
 // Addressing/epilogue modes of the kernel.
 enum Mode : int {
@@ -133,18 +105,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                           const __grid_constant__ CUtensorMap tm_q16,
                           const __grid_constant__ CUtensorMap tm_k16,
                           const __grid_constant__ CUtensorMap tm_v16, void* __restrict__ out,
-                          float* __restrict__ lse, int Bn, int H, int Sq, int Skv,
-                          float scale_log2, float rescale_log2, int s_local, int n_split,
-                          int n_items, int* err, long long wait_limit) {
+                          float* __restrict__ lse, int H, int Sq, int Skv, float scale_log2,
+                          float rescale_log2, int s_local, int n_split, int b_first, int n_full,
+                          int n_tail, int tail_parts, float* __restrict__ ws_o,
+                          float* __restrict__ ws_lse, int* err, long long wait_limit) {
   using G = Geometry<D>;
   constexpr bool kAcc = kMode == kAccum;
-  // kSharded: the DeepSpeed Ulysses path in one kernel.  The item's batch index is the head
-  // group g (P of them), its head index the head j inside it (H = heads per group); head
-  // g*H + j of the full sequence is read straight from the sequence shards [P][S_l][H*P][D]
-  // (token t lives in shard t / S_l, row t % S_l), and O goes back to the same sharded
-  // layout: the all-to-alls become addressing.  A tile inside one shard is a single
-  // 128-row box (tm_q/k/v); a tile that straddles a shard boundary is eight 16-row boxes
-  // (tm_q16/k16/v16; S_l % 16 == 0, so no box crosses a boundary).
+  // kSharded: the DeepSpeed Ulysses path in one kernel.  The grid's z is the head group g
+  // (P of them), y the head j inside it (H = heads per group); head g*H + j of the full
+  // sequence is read straight from the sequence shards [P][S_l][H*P][D] (token t lives in
+  // shard t / S_l, row t % S_l) with 16-row TMA boxes, so no box crosses a shard boundary
+  // (S_l % 16 == 0), and O goes back to the same sharded layout: the all-to-alls become
+  // addressing.  A tile inside one shard is a single 128-row box (tm_q/k/v); only tiles
+  // that straddle a shard boundary use the 16-row maps (tm_q16/k16/v16).
   constexpr bool kShard = kMode == kSharded;
   extern __shared__ uint8_t smem_raw[];
   __shared__ Barriers bars;
@@ -156,14 +129,49 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t smem_base = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n_pairs = (Sq + 2 * kBlockM - 1) / (2 * kBlockM);
+  int pair, h, b, split, n_ranges;
+  int slot = -1;  // tail split: this CTA's workspace slot (-1: writes the output itself)
+  if (n_full < 0) {
+    // 3-D grid.  split-KV: blockIdx.x = (query tile pair) * n_split + split; range `split`
+    // writes its partial (O, LSE) to its own slice of out / lse
+    split = n_split > 1 ? int(blockIdx.x % unsigned(n_split)) : 0;
+    n_ranges = n_split;
+    pair = int(blockIdx.x / unsigned(n_split));
+    h = blockIdx.y;
+    b = b_first + int(blockIdx.z);
+    if (n_split > 1) {
+      out = static_cast<char*>(out) + size_t(split) * gridDim.z * Sq * H * D * (kOutF32 ? 4 : 2);
+      lse += size_t(split) * gridDim.z * H * Sq;
+    }
+  } else {
+    // 1-D grid: whole items first, then the tail items' key ranges (items numbered tile
+    // pair fastest, then head, then batch)
+    const int x = int(blockIdx.x);
+    int item = x;
+    split = 0;
+    n_ranges = 1;
+    if (x >= n_full) {
+      const int t = (x - n_full) / tail_parts;
+      split = (x - n_full) - t * tail_parts;
+      n_ranges = tail_parts;
+      item = n_full + t;
+      slot = split * n_tail + t;
+    }
+    const int n_pairs = (Sq + 2 * kBlockM - 1) / (2 * kBlockM);
+    pair = item % n_pairs;
+    h = (item / n_pairs) % H;
+    b = b_first + item / n_pairs / H;
+  }
+  const int q_first = pair * (2 * kBlockM);
+  const int head_coord = kShard ? b * H + h : h;  // head coordinate in the tensor maps
   const int n_kv_all = (Skv + kBlockN - 1) / kBlockN;
-  const int item_first = int(blockIdx.x), item_step = int(gridDim.x);
+  const int kv_base = n_kv_all / n_ranges, kv_rem = n_kv_all % n_ranges;
+  const int j0 = split * kv_base + (split < kv_rem ? split : kv_rem);  // first key block
+  const int n_kv = kv_base + (split < kv_rem ? 1 : 0);                 // key blocks here
   volatile int* abort_flag = &abort_sh;
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&bars.q_full), 1);
-    mbar_init(smem_u32(&bars.q_empty), 1);
     for (int s = 0; s < kSlots; ++s) {
       mbar_init(smem_u32(&bars.full[s]), 1);
       mbar_init(smem_u32(&bars.empty[s]), 1);
@@ -172,9 +180,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&bars.s_full[t]), 1);
       for (int c = 0; c < kPChunks; ++c)
         mbar_init(smem_u32(&bars.p_part[t][c]), 4);  // one arrive per softmax warp
-      mbar_init(smem_u32(&bars.o_full[t]), 1);
-      mbar_init(smem_u32(&bars.o_empty[t]), 4);    // one arrive per softmax warp
     }
+    mbar_init(smem_u32(&bars.o_full), 1);
     mbar_init(smem_u32(&bars.drain), 1);
     abort_sh = 0;
     fence_mbar_init();
@@ -197,6 +204,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  // The launch is a dependent one: the set-up above may overlap the previous kernel's last
+  // wave, nothing below reads or writes global memory before that kernel has completed, and
+  // the next kernel may be scheduled from here on (it waits the same way).
+  griddep_wait();
+  griddep_release();
 
   if (warp < 8) {
     // ------------------------------------------------------------------ softmax warps
@@ -209,222 +221,245 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_o = tmem + lane_bits + uint32_t(2 * kBlockN + tile * D);
     const uint32_t bar_s = smem_u32(&bars.s_full[tile]);
     const uint32_t bar_p0 = smem_u32(&bars.p_part[tile][0]);  // chunk c at + 8 c
+    float m = -INFINITY;  // running (possibly stale) max of x = s * scale * log2(e)
+    float l = 0.f;        // running sum of 2^(x - m)
     bool ok = true;
-    uint32_t blk = 0;  // key blocks of all items so far: the s_full / p_part phase
 
-    for (int item = item_first, it = 0; ok && item < n_items; item += item_step, ++it) {
-      int j0, n_kv;
-      key_range(decode_item(item, n_pairs, n_split, H).split, n_split, n_kv_all, j0, n_kv);
-      float m = -INFINITY;  // running max of x = s * scale * log2(e)
-      float l = 0.f;        // running sum of 2^(x - m)
-
-      for (int j = 0; j < n_kv; ++j, ++blk) {
-        ok = mbar_wait(bar_s, blk & 1u, abort_flag, err, wait_limit);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        tc_fence_after();
-
-        float x[kBlockN];
-        {
-          uint32_t r[kBlockN];
-          tmem_ld128(t_s, r);  // the whole S row, one wait
-#pragma unroll
-          for (int c = 0; c < kBlockN; ++c) x[c] = __uint_as_float(r[c]);
-        }
-        const int valid = Skv - (j0 + j) * kBlockN;  // keys of this block inside the sequence
-        if (valid < kBlockN) {
-#pragma unroll
-          for (int c = 0; c < kBlockN; ++c)
-            if (c >= valid) x[c] = -INFINITY;
-        }
-        // row maximum of the raw logits (scale > 0 is a precondition of the call): a tree
-        // of three-input max, 64 instructions and 5 levels deep (a chain would be
-        // latency-bound)
-        float mx;
-        {
-          float l1[44];
-#pragma unroll
-          for (int i = 0; i < 42; ++i) l1[i] = max3(x[3 * i], x[3 * i + 1], x[3 * i + 2]);
-          l1[42] = x[126];
-          l1[43] = x[127];
-          float l2[16];
-#pragma unroll
-          for (int i = 0; i < 14; ++i) l2[i] = max3(l1[3 * i], l1[3 * i + 1], l1[3 * i + 2]);
-          l2[14] = l1[42];
-          l2[15] = l1[43];
-          float l3[6];
-#pragma unroll
-          for (int i = 0; i < 5; ++i) l3[i] = max3(l2[3 * i], l2[3 * i + 1], l2[3 * i + 2]);
-          l3[5] = l2[15];
-          mx = fmaxf(max3(l3[0], l3[1], l3[2]), max3(l3[3], l3[4], l3[5]));
-        }
-        const float m_tile = mx * scale_log2;
-        float alpha = 1.0f;
-        bool rescale = false;
-        if (j == 0) {
-          m = m_tile;
-        } else {
-          const bool grow = m_tile > m + rescale_log2;
-          rescale = __any_sync(0xffffffffu, grow);
-          if (rescale) {
-            const float m_new = grow ? m_tile : m;
-            alpha = ex2(m - m_new);
-            m = m_new;
-            l *= alpha;
-          }
-        }
-        // p = 2^(x * scale_log2 - m): most pairs on the special-function unit, kPolyPairs
-        // of every 8 pairs on the FMA pipe (exp2_poly2); p rounded to bf16 for the PV
-        // product and written over S as bf16 pairs; the row sum keeps the unrounded fp32
-        // p.  The keys go in kPChunks chunks with one handoff each, so that the issuer runs
-        // O += P V of the first chunks while the rest of P is computed.
-        const float2 sl2 = make_float2(scale_log2, scale_log2);
-        const float2 nm2 = make_float2(-m, -m);
-        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int part = 0; part < kPChunks; ++part) {
-          uint32_t pk[kChunkPairs];
-#pragma unroll
-          for (int e = 0; e < kChunkPairs; ++e) {
-            const int c = 2 * (part * kChunkPairs + e);
-            const float2 t = ffma2(make_float2(x[c], x[c + 1]), sl2, nm2);
-            float2 pv;
-            if ((e & 7) >= 8 - kPolyPairs) {
-              pv = exp2_poly2(t);
-            } else {
-              pv.x = ex2(t.x);
-              pv.y = ex2(t.y);
-            }
-            if (e & 1) acc1 = fadd2(acc1, pv);
-            else acc0 = fadd2(acc0, pv);
-            pk[e] = pack_bf16x2(pv.x, pv.y);
-          }
-          tmem_st_any(t_s + part * kChunkPairs, pk);
-          if (part == 0 && rescale) {
-            // rescale this warp's O rows by alpha before the first PV chunk accumulates
-            // into them: PV of the previous block has completed (the issuer committed this
-            // block's S after it), and no PV of this block starts before the arrive below
-            const float2 a2 = make_float2(alpha, alpha);
-#pragma unroll
-            for (int oc = 0; oc < D / 32; ++oc) {
-              uint32_t r[32];
-              tmem_ld32(t_o + oc * 32, r);
-#pragma unroll
-              for (int c = 0; c < 32; c += 2) {
-                const float2 o =
-                    fmul2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), a2);
-                r[c] = __float_as_uint(o.x);
-                r[c + 1] = __float_as_uint(o.y);
-              }
-              tmem_st32(t_o + oc * 32, r);
-            }
-          }
-          // hand this chunk over: every lane's TMEM stores complete, then one arrive per warp
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar_p0 + 8 * part);
-        }
-        const float2 acc = fadd2(acc0, acc1);
-        l += acc.x + acc.y;
-      }
-      if (!ok) break;
-
-      // ---------------------------------------------------------------- epilogue
-      ok = mbar_wait(smem_u32(&bars.o_full[tile]), uint32_t(it) & 1u, abort_flag, err,
-                     wait_limit);
+    for (int j = 0; j < n_kv; ++j) {
+      ok = mbar_wait(bar_s, j & 1, abort_flag, err, wait_limit);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      const Item wi = decode_item(item, n_pairs, n_split, H);  // (not kept live over the loop)
-      // split-KV: key range s writes its partial (O, LSE) to its own slice of out / lse
-      float* lse_it = lse;
-      char* out_it = static_cast<char*>(out);
-      if (n_split > 1) {
-        out_it += size_t(wi.split) * Bn * Sq * H * D * (kOutF32 ? 4 : 2);
-        lse_it += size_t(wi.split) * Bn * H * Sq;
+
+      float x[kBlockN];
+      {
+        uint32_t r[kBlockN];
+        tmem_ld128(t_s, r);  // the whole S row, one wait
+#pragma unroll
+        for (int c = 0; c < kBlockN; ++c) x[c] = __uint_as_float(r[c]);
       }
-      const int head_coord = kShard ? wi.b * H + wi.h : wi.h;
-      const int q = wi.pair * (2 * kBlockM) + tile * kBlockM + row;
-      const bool in_range = q < Sq;
-      const int qr = in_range ? q : 0;
-      // sharded layout: token q = r * S_l + s sits at row q of the flattened [P][S_l] shards
-      const size_t row_off = kShard ? (size_t(qr) * (H * Bn) + head_coord) * size_t(D)
-                                    : ((size_t(wi.b) * Sq + qr) * H + wi.h) * size_t(D);
-      const size_t lse_idx = (size_t(wi.b) * H + wi.h) * Sq + qr;
-      // this item's result: O_c = O_tmem / l, LSE_c = ln(2^m * l) = (m + log2 l) * ln 2
+      const int valid = Skv - (j0 + j) * kBlockN;  // keys of this block inside the sequence
+      if (valid < kBlockN) {
+#pragma unroll
+        for (int c = 0; c < kBlockN; ++c)
+          if (c >= valid) x[c] = -INFINITY;
+      }
+      // row maximum of the raw logits (scale > 0 is a precondition of the call): a tree of
+      // three-input max, 64 instructions and 5 levels deep (a chain would be latency-bound)
+      float mx;
+      {
+        float l1[44];
+#pragma unroll
+        for (int i = 0; i < 42; ++i) l1[i] = max3(x[3 * i], x[3 * i + 1], x[3 * i + 2]);
+        l1[42] = x[126];
+        l1[43] = x[127];
+        float l2[16];
+#pragma unroll
+        for (int i = 0; i < 14; ++i) l2[i] = max3(l1[3 * i], l1[3 * i + 1], l1[3 * i + 2]);
+        l2[14] = l1[42];
+        l2[15] = l1[43];
+        float l3[6];
+#pragma unroll
+        for (int i = 0; i < 5; ++i) l3[i] = max3(l2[3 * i], l2[3 * i + 1], l2[3 * i + 2]);
+        l3[5] = l2[15];
+        mx = fmaxf(max3(l3[0], l3[1], l3[2]), max3(l3[3], l3[4], l3[5]));
+      }
+      const float m_tile = mx * scale_log2;
+      float alpha = 1.0f;
+      bool rescale = false;
+      if (j == 0) {
+        m = m_tile;
+      } else {
+        const bool grow = m_tile > m + rescale_log2;
+        rescale = __any_sync(0xffffffffu, grow);
+        if (rescale) {
+          const float m_new = grow ? m_tile : m;
+          alpha = ex2(m - m_new);
+          m = m_new;
+          l *= alpha;
+        }
+      }
+      // p = 2^(x * scale_log2 - m): most pairs on the special-function unit, kPolyPairs of
+      // every 8 pairs on the FMA pipe (exp2_poly2); p rounded to bf16 for the PV product and
+      // written over S as bf16 pairs; the row sum keeps the unrounded fp32 p.  The keys go
+      // in kPChunks chunks with one handoff each, so that the issuer runs O += P V of the
+      // first chunks while the rest of P is computed.
+      const float2 sl2 = make_float2(scale_log2, scale_log2);
+      const float2 nm2 = make_float2(-m, -m);
+      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int part = 0; part < kPChunks; ++part) {
+        uint32_t pk[kChunkPairs];
+#pragma unroll
+        for (int e = 0; e < kChunkPairs; ++e) {
+          const int c = 2 * (part * kChunkPairs + e);
+          const float2 t = ffma2(make_float2(x[c], x[c + 1]), sl2, nm2);
+          float2 pv;
+          if ((e & 7) >= 8 - kPolyPairs) {
+            pv = exp2_poly2(t);
+          } else {
+            pv.x = ex2(t.x);
+            pv.y = ex2(t.y);
+          }
+          if (e & 1) acc1 = fadd2(acc1, pv);
+          else acc0 = fadd2(acc0, pv);
+          pk[e] = pack_bf16x2(pv.x, pv.y);
+        }
+        tmem_st_any(t_s + part * kChunkPairs, pk);
+        if (part == 0 && rescale) {
+          // rescale this warp's O rows by alpha before the first PV chunk accumulates into
+          // them: PV of the previous block has completed (the issuer committed this
+          // block's S after it), and no PV of this block starts before the arrive below
+          const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+          for (int oc = 0; oc < D / 32; ++oc) {
+            uint32_t r[32];
+            tmem_ld32(t_o + oc * 32, r);
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+              const float2 o =
+                  fmul2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), a2);
+              r[c] = __float_as_uint(o.x);
+              r[c + 1] = __float_as_uint(o.y);
+            }
+            tmem_st32(t_o + oc * 32, r);
+          }
+        }
+        // hand this chunk over: every lane's TMEM stores complete, then one arrive per warp
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_p0 + 8 * part);
+      }
+      const float2 acc = fadd2(acc0, acc1);
+      l += acc.x + acc.y;
+    }
+
+    // ------------------------------------------------------------------ epilogue
+    const int q = q_first + tile * kBlockM + row;
+    const bool in_range = q < Sq;
+    const int qr = in_range ? q : 0;
+    // sharded layout: token q = r * S_l + s sits at row q of the flattened [P][S_l] shards
+    // (P = Sq / S_l head groups in all, whichever of them this launch covers)
+    const size_t row_off = kShard ? (size_t(qr) * (H * (Sq / s_local)) + head_coord) * size_t(D)
+                                  : ((size_t(b) * Sq + qr) * H + h) * size_t(D);
+    const size_t lse_idx = (size_t(b) * H + h) * Sq + (in_range ? q : 0);
+    // bf16 accumulate: the running row and its LSE are loaded now, before the last
+    // O += P V has completed, so that one memory round trip overlaps it instead of one per
+    // 32-column chunk after it.  (An empty accumulator's row may hold anything: it is
+    // loaded but never used.)
+    constexpr bool kPreload = kAcc && !kOutF32;
+    uint4 acc_row[kPreload ? D / 8 : 1];
+    float la_pre = -INFINITY;
+    if constexpr (kPreload) {
+      if (ok && slot < 0 && in_range) {
+        la_pre = lse[lse_idx];
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(out) + row_off);
+#pragma unroll
+        for (int e = 0; e < D / 8; ++e) acc_row[e] = src[e];
+      }
+    }
+    if (ok) {
+      ok = mbar_wait(smem_u32(&bars.o_full), 0, abort_flag, err, wait_limit);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      // this block's result: O_c = O_tmem / l, LSE_c = ln(2^m * l) = (m + log2 l) * ln 2
       const float lc2 = m + log2f(l);  // LSE_c in base 2
       float fa = 0.f, fc = 1.0f / l;   // written row = fa * O_acc + fc * O_tmem
       float lse_out = lc2 * kLn2;
+      if (slot >= 0) {
+        // tail split: the normalised partial of this key range, fp32, to workspace row
+        // (slot, tile * 128 + row); the combine kernel folds the ranges afterwards
+        const size_t wrow = size_t(slot) * (2 * kBlockM) + tile * kBlockM + row;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(t_o + c * 32, r);
+          if (in_range) {
+            float4* dst = reinterpret_cast<float4*>(ws_o + wrow * D + c * 32);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(r[4 * e]) * fc, __uint_as_float(r[4 * e + 1]) * fc,
+                                   __uint_as_float(r[4 * e + 2]) * fc, __uint_as_float(r[4 * e + 3]) * fc);
+          }
+        }
+        if (in_range) ws_lse[wrow] = lse_out;
+      } else {
       if constexpr (kAcc) {
         // Ring Attention step fused into the epilogue: merge (O_c, LSE_c) into the running
         // (O_acc, LSE_acc) in place; an empty accumulator (LSE_acc = -inf) takes O_c
         if (in_range) {
-          const float la2 = lse_it[lse_idx] * kLog2e;
-          const float mxl = fmaxf(la2, lc2);
-          const float wa = exp2f(la2 - mxl), wc = exp2f(lc2 - mxl);
+          const float la2 = (kPreload ? la_pre : lse[lse_idx]) * kLog2e;
+          const float mx = fmaxf(la2, lc2);
+          const float wa = exp2f(la2 - mx), wc = exp2f(lc2 - mx);
           const float tot = wa + wc;
           fa = wa / tot;
           fc = wc / (tot * l);
-          lse_out = (mxl + log2f(tot)) * kLn2;
+          lse_out = (mx + log2f(tot)) * kLn2;
         }
       }
-      // O in 32-column chunks: TMEM -> registers -> scaled (and merged) -> global.  After
-      // the last chunk's TMEM load the warp releases O, so that the issuer may start the
-      // next item's O += P V into these columns while the last chunk is stored.
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(t_o + c * 32, r);
-        if (c == D / 32 - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&bars.o_empty[tile]));
-        }
-        if (in_range) {
-          if constexpr (kOutF32) {
-            float4* dst =
-                reinterpret_cast<float4*>(reinterpret_cast<float*>(out_it) + row_off + c * 32);
+      // one 32-column chunk of the row: scaled (and merged into the accumulator) and stored
+      auto store_chunk = [&](int c, const uint32_t (&r)[32]) {
+        if (!in_range) return;
+        if constexpr (kOutF32) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + row_off + c * 32);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              float4 v = make_float4(__uint_as_float(r[4 * e]) * fc, __uint_as_float(r[4 * e + 1]) * fc,
-                                     __uint_as_float(r[4 * e + 2]) * fc, __uint_as_float(r[4 * e + 3]) * fc);
-              if (kAcc && fa != 0.f) {  // an empty accumulator row is never read
-                const float4 a = dst[e];
-                v.x = fmaf(fa, a.x, v.x);
-                v.y = fmaf(fa, a.y, v.y);
-                v.z = fmaf(fa, a.z, v.z);
-                v.w = fmaf(fa, a.w, v.w);
-              }
-              dst[e] = v;
+          for (int e = 0; e < 8; ++e) {
+            float4 v = make_float4(__uint_as_float(r[4 * e]) * fc, __uint_as_float(r[4 * e + 1]) * fc,
+                                   __uint_as_float(r[4 * e + 2]) * fc, __uint_as_float(r[4 * e + 3]) * fc);
+            if (kAcc && fa != 0.f) {  // an empty accumulator row is never read
+              const float4 a = dst[e];
+              v.x = fmaf(fa, a.x, v.x);
+              v.y = fmaf(fa, a.y, v.y);
+              v.z = fmaf(fa, a.z, v.z);
+              v.w = fmaf(fa, a.w, v.w);
             }
-          } else {
-            uint4* dst =
-                reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(out_it) + row_off + c * 32);
+            dst[e] = v;
+          }
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + row_off + c * 32);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float o[8];
+          for (int e = 0; e < 4; ++e) {
+            float o[8];
 #pragma unroll
-              for (int t = 0; t < 8; ++t) o[t] = __uint_as_float(r[8 * e + t]) * fc;
-              if (kAcc && fa != 0.f) {  // an empty accumulator row is never read
-                const uint4 a = dst[e];
-                const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+            for (int t = 0; t < 8; ++t) o[t] = __uint_as_float(r[8 * e + t]) * fc;
+            if (kAcc && fa != 0.f) {  // an empty accumulator's row is not used
+              uint4 a;
+              if constexpr (kPreload) a = acc_row[c * 4 + e];
+              else a = dst[e];
+              const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                  o[2 * t] = fmaf(fa, __uint_as_float(aw[t] << 16), o[2 * t]);
-                  o[2 * t + 1] = fmaf(fa, __uint_as_float(aw[t] & 0xFFFF0000u), o[2 * t + 1]);
-                }
+              for (int t = 0; t < 4; ++t) {
+                o[2 * t] = fmaf(fa, __uint_as_float(aw[t] << 16), o[2 * t]);
+                o[2 * t + 1] = fmaf(fa, __uint_as_float(aw[t] & 0xFFFF0000u), o[2 * t + 1]);
               }
-              uint4 v;
-              v.x = pack_bf16x2(o[0], o[1]);
-              v.y = pack_bf16x2(o[2], o[3]);
-              v.z = pack_bf16x2(o[4], o[5]);
-              v.w = pack_bf16x2(o[6], o[7]);
-              dst[e] = v;
             }
+            uint4 v;
+            v.x = pack_bf16x2(o[0], o[1]);
+            v.y = pack_bf16x2(o[2], o[3]);
+            v.z = pack_bf16x2(o[4], o[5]);
+            v.w = pack_bf16x2(o[6], o[7]);
+            dst[e] = v;
           }
         }
+      };
+      if constexpr (kPreload) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {  // unrolled: acc_row is indexed statically
+          uint32_t r[32];
+          tmem_ld32(t_o + c * 32, r);
+          store_chunk(c, r);
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(t_o + c * 32, r);
+          store_chunk(c, r);
+        }
       }
-      if (in_range) {
-        if (lse_it != nullptr) lse_it[lse_idx] = lse_out;
+      if (in_range && lse != nullptr) lse[lse_idx] = lse_out;
       }
     }
   } else {
@@ -434,9 +469,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------ TMA producer
     if (elect_one()) {
       // one 128-row tile starting at token t0 into `dst`: a 64-column box per 128-byte
-      // column block; sharded inputs take eight 16-row boxes when the tile crosses shards
+      // column block; sharded inputs take eight 16-row boxes, each inside one rank shard
       auto load_tile = [&](const CUtensorMap* map, const CUtensorMap* map16, uint32_t dst,
-                           uint32_t bar, int t0, int head_coord, int b) {
+                           uint32_t bar, int t0) {
         if constexpr (!kShard) {
 #pragma unroll
           for (int bx = 0; bx < G::kBoxes; ++bx)
@@ -465,43 +500,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
       const uint32_t bar_q = smem_u32(&bars.q_full);
-      int issued = 0;    // ring uses issued (K and V tiles)
-      int q_issued = 0;  // items whose Q load was issued
-      bool ok = true;
-      for (int item = item_first, it = 0; ok && item < n_items; item += item_step, ++it) {
-        const Item wi = decode_item(item, n_pairs, n_split, H);
-        int j0, n_kv;
-        key_range(wi.split, n_split, n_kv_all, j0, n_kv);
-        const int head_coord = kShard ? wi.b * H + wi.h : wi.h;
-        const int b_coord = kShard ? 0 : wi.b;
-        // the previous item's last Q K^T has read Q before it is overwritten
-        if (it > 0 && !(ok = mbar_wait(smem_u32(&bars.q_empty), uint32_t(it - 1) & 1u,
-                                       abort_flag, err, wait_limit)))
-          break;
-        mbar_arrive_expect_tx(bar_q, 2 * G::kTileBytes);
+      mbar_arrive_expect_tx(bar_q, 2 * G::kTileBytes);
 #pragma unroll
-        for (int t = 0; t < 2; ++t)
-          load_tile(&tm_q, &tm_q16, smem_base + G::kOffQ + t * G::kTileBytes, bar_q,
-                    wi.pair * (2 * kBlockM) + t * kBlockM, head_coord, b_coord);
-        q_issued = it + 1;
-        for (int u = 0; u < 2 * n_kv; ++u) {
-          const int use = issued;
-          const int slot = use % kSlots;
-          const uint32_t ph = uint32_t(use / kSlots) & 1u;
-          if (!(ok = mbar_wait(smem_u32(&bars.empty[slot]), ph ^ 1u, abort_flag, err,
-                               wait_limit)))
-            break;
-          const uint32_t bar_f = smem_u32(&bars.full[slot]);
-          mbar_arrive_expect_tx(bar_f, G::kTileBytes);
-          load_tile((u & 1) ? &tm_v : &tm_k, (u & 1) ? &tm_v16 : &tm_k16,
-                    smem_base + G::kOffSlots + slot * G::kTileBytes, bar_f,
-                    (j0 + (u >> 1)) * kBlockN, head_coord, b_coord);
-          issued = use + 1;
-        }
+      for (int t = 0; t < 2; ++t)
+        load_tile(&tm_q, &tm_q16, smem_base + G::kOffQ + t * G::kTileBytes, bar_q,
+                  q_first + t * kBlockM);
+      int issued = 0;
+      for (int use = 0; use < 2 * n_kv; ++use) {
+        const int slot = use % kSlots;
+        const uint32_t ph = uint32_t(use / kSlots) & 1u;
+        if (!mbar_wait(smem_u32(&bars.empty[slot]), ph ^ 1u, abort_flag, err, wait_limit)) break;
+        const uint32_t bar_f = smem_u32(&bars.full[slot]);
+        mbar_arrive_expect_tx(bar_f, G::kTileBytes);
+        load_tile((use & 1) ? &tm_v : &tm_k, (use & 1) ? &tm_v16 : &tm_k16,
+                  smem_base + G::kOffSlots + slot * G::kTileBytes, bar_f,
+                  (j0 + (use >> 1)) * kBlockN);
+        issued = use + 1;
       }
       // drain: every issued copy must have landed before the CTA's shared memory is
       // released (immediate on the normal path, where the consumer already saw them)
-      if (q_issued > 0) drain_wait(bar_q, uint32_t(q_issued - 1) & 1u, wait_limit);
+      drain_wait(bar_q, 0, wait_limit);
       for (int use = issued - kSlots < 0 ? 0 : issued - kSlots; use < issued; ++use)
         drain_wait(smem_u32(&bars.full[use % kSlots]), uint32_t(use / kSlots) & 1u, wait_limit);
     }
@@ -518,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // S_t = Q_t K^T over D in K=16 steps; K-major 128-B swizzled operands: 32 B per
       // step inside a 128-B row, the next 64 columns in the next box
       auto issue_qk = [&](int t, uint32_t k_addr) {
-#pragma unroll 4
+#pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * G::kBoxBytes + (kk & 3) * 32;
           mma_ss(t_s[t], sdesc_sw128(q_addr[t] + off, 16, 1024),
@@ -538,16 +556,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto slot_addr = [&](int use) {
         return smem_base + G::kOffSlots + (use % kSlots) * G::kTileBytes;
       };
-      // O_t += P_t V, chunk by chunk as the softmax warps hand P over (first block of an
-      // item: the accumulator starts from zero)
-      auto issue_pv = [&](int t, uint32_t v_addr, bool first, uint32_t blk) {
+      // O_t += P_t V, chunk by chunk as the softmax warps hand P over
+      auto issue_pv = [&](int t, uint32_t v_addr, int j) {
 #pragma unroll
         for (int part = 0; part < kPChunks; ++part) {
-          if (!mbar_wait(smem_u32(&bars.p_part[t][part]), blk & 1u, abort_flag, err,
+          if (!mbar_wait(smem_u32(&bars.p_part[t][part]), uint32_t(j) & 1u, abort_flag, err,
                          wait_limit))
             return false;
           tc_fence_after();
-          issue_pv_chunk(t, v_addr, !first || part > 0, part);
+          issue_pv_chunk(t, v_addr, j > 0 || part > 0, part);
         }
         return true;
       };
@@ -556,64 +573,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                          abort_flag, err, wait_limit);
       };
 
-      bool ok = true;
-      int use = 0;       // ring uses consumed so far
-      uint32_t blk = 0;  // key blocks of all items so far
-      for (int item = item_first, it = 0; ok && item < n_items; item += item_step, ++it) {
-        const Item wi = decode_item(item, n_pairs, n_split, H);
-        int j0, n_kv;
-        key_range(wi.split, n_split, n_kv_all, j0, n_kv);
-        // first S of the item: Q landed and K_0 in the ring.  S_t of this item overwrites
-        // P_t of the previous one only after that item's last O += P V (issue order).
-        if (!(ok = mbar_wait(smem_u32(&bars.q_full), uint32_t(it) & 1u, abort_flag, err,
-                             wait_limit) && wait_full(use)))
-          break;
+      bool ok = mbar_wait(smem_u32(&bars.q_full), 0, abort_flag, err, wait_limit) && wait_full(0);
+      if (ok) {
         tc_fence_after();
-        issue_qk(0, slot_addr(use));
+        issue_qk(0, slot_addr(0));
         tc_commit(smem_u32(&bars.s_full[0]));
-        issue_qk(1, slot_addr(use));
+        issue_qk(1, slot_addr(0));
         tc_commit(smem_u32(&bars.s_full[1]));
-        tc_commit(smem_u32(&bars.empty[use % kSlots]));
-        if (n_kv == 1) tc_commit(smem_u32(&bars.q_empty));
-        ++use;
-        for (int j = 0; j < n_kv; ++j, ++blk) {
-          const int use_v = use, use_k = use + 1;
-          const bool more = j + 1 < n_kv;
-          if (!(ok = wait_full(use_v))) break;
-          if (j == 0 && it > 0) {
-            // O_0 is overwritten by this item's first O += P V: the softmax warps have read
-            // the previous item's O out of it
-            if (!(ok = mbar_wait(smem_u32(&bars.o_empty[0]), uint32_t(it - 1) & 1u, abort_flag,
-                                 err, wait_limit)))
-              break;
-            tc_fence_after();
-          }
-          if (!(ok = issue_pv(0, slot_addr(use_v), j == 0, blk))) break;
-          if (!more) tc_commit(smem_u32(&bars.o_full[0]));
-          if (more) {
-            if (!(ok = wait_full(use_k))) break;
-            tc_fence_after();
-            issue_qk(0, slot_addr(use_k));
-            tc_commit(smem_u32(&bars.s_full[0]));
-          }
-          if (j == 0 && it > 0) {
-            if (!(ok = mbar_wait(smem_u32(&bars.o_empty[1]), uint32_t(it - 1) & 1u, abort_flag,
-                                 err, wait_limit)))
-              break;
-            tc_fence_after();
-          }
-          if (!(ok = issue_pv(1, slot_addr(use_v), j == 0, blk))) break;
-          tc_commit(smem_u32(&bars.empty[use_v % kSlots]));
-          if (!more) tc_commit(smem_u32(&bars.o_full[1]));
-          if (more) {
-            issue_qk(1, slot_addr(use_k));
-            tc_commit(smem_u32(&bars.s_full[1]));
-            tc_commit(smem_u32(&bars.empty[use_k % kSlots]));
-            if (j + 2 == n_kv) tc_commit(smem_u32(&bars.q_empty));  // the item's last Q K^T
-          }
-          use += more ? 2 : 1;
+        tc_commit(smem_u32(&bars.empty[0]));
+      }
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int use_v = 2 * j + 1, use_k = 2 * j + 2;
+        const bool more = j + 1 < n_kv;
+        if (!(ok = wait_full(use_v))) break;
+        if (!(ok = issue_pv(0, slot_addr(use_v), j))) break;
+        if (more) {
+          if (!(ok = wait_full(use_k))) break;
+          tc_fence_after();
+          issue_qk(0, slot_addr(use_k));
+          tc_commit(smem_u32(&bars.s_full[0]));
+        }
+        if (!(ok = issue_pv(1, slot_addr(use_v), j))) break;
+        tc_commit(smem_u32(&bars.empty[use_v % kSlots]));
+        if (more) {
+          issue_qk(1, slot_addr(use_k));
+          tc_commit(smem_u32(&bars.s_full[1]));
+          tc_commit(smem_u32(&bars.empty[use_k % kSlots]));
         }
       }
+      if (ok) tc_commit(smem_u32(&bars.o_full));
       // drain: no MMA may still be writing TMEM when it is freed
       tc_commit(smem_u32(&bars.drain));
       drain_wait(smem_u32(&bars.drain), 0, wait_limit);
@@ -627,9 +615,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kWarpMma) tmem_dealloc(tmem, kTmemCols);
 }
 
-// Launch geometry shared by every mode: n_items work items over at most one CTA per SM.
+// Launch arguments shared by every mode and grid form.
 struct Launch {
-  int Bn, H, Sq, Skv, s_local, n_split, n_items;
+  dim3 grid;
+  int H, Sq, Skv, s_local, n_split, b_first;
+  int n_full, n_tail, tail_parts;  // n_full < 0: 3-D grid form
+  float* ws_o;
+  float* ws_lse;
   float scale_log2, rescale_log2;
   int* err;
   long long wait_limit;
@@ -644,13 +636,21 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        G::kDynSmem);
   if (e != cudaSuccess) return e;
-  const int sms = sm_count();
-  const unsigned grid = unsigned(a.n_items < sms ? a.n_items : sms);
-  kernel<<<grid, kThreads, G::kDynSmem, stream>>>(tq, tk, tv, tq16, tk16, tv16, out, lse, a.Bn,
-                                                   a.H, a.Sq, a.Skv, a.scale_log2,
-                                                   a.rescale_log2, a.s_local, a.n_split,
-                                                   a.n_items, a.err, a.wait_limit);
-  return cudaGetLastError();
+  // launched as a dependent of the previous kernel on the stream (see griddep_wait)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = a.grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = G::kDynSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, tq, tk, tv, tq16, tk16, tv16, out, lse, a.H, a.Sq, a.Skv,
+                            a.scale_log2, a.rescale_log2, a.s_local, a.n_split, a.b_first,
+                            a.n_full, a.n_tail, a.tail_parts, a.ws_o, a.ws_lse, a.err,
+                            a.wait_limit);
 }
 
 template <int D, int kMode>
@@ -686,30 +686,82 @@ cudaError_t launch_any(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
 
 }  // namespace
 
+TailSplit tail_split_plan(int B, int H, int Sq, int Skv) {
+  TailSplit t{};
+  const long long pairs = (Sq + 2 * kBlockM - 1) / (2 * kBlockM);
+  const long long items = pairs * H * B;
+  const int sms = sm_count();
+  const int n_kv = (Skv + kBlockN - 1) / kBlockN;
+  if (items < 1 || items > 0x7fffffffLL || n_kv < 2) return t;
+  const long long rem = items % sms;  // items of the last, partial wave
+  if (rem == 0) return t;
+  // split each of them into as many key ranges as still fit in one wave (at most 8, and
+  // at least 2 key blocks per range)
+  long long parts = sms / rem;
+  if (parts > 8) parts = 8;
+  if (parts > n_kv / 2) parts = n_kv / 2;
+  if (parts < 2) return t;
+  t.n_full = int(items - rem);
+  t.n_tail = int(rem);
+  t.parts = int(parts);
+  return t;
+}
+
+size_t tail_split_workspace(const TailSplit& t, int D) {
+  if (t.parts < 2) return 0;
+  const size_t rows = size_t(t.parts) * t.n_tail * (2 * kBlockM);
+  return ((rows * D * 4 + 255) & ~size_t(255)) + rows * 4;
+}
+
 cudaError_t launch_attn_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
                                   const CUtensorMap& tv, void* out, float* lse, int B, int H,
                                   int Sq, int Skv, int D, float scale_log2, float rescale_log2,
                                   bool out_f32, bool accumulate, int n_split, int* err,
                                   long long wait_limit, cudaStream_t stream) {
-  const long long n_items = (long long)((Sq + 2 * kBlockM - 1) / (2 * kBlockM)) * n_split * H * B;
-  if (n_items > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  const Launch a{B, H, Sq, Skv, 0, n_split, int(n_items), scale_log2, rescale_log2, err,
-                 wait_limit};
-  return launch_any(tq, tk, tv, tq, tk, tv, out, lse, D, a, out_f32,
-                    accumulate ? kAccum : kPlain, stream);
+  Launch a{};
+  a.grid = dim3(((Sq + 2 * kBlockM - 1) / (2 * kBlockM)) * n_split, H, B);
+  a.H = H, a.Sq = Sq, a.Skv = Skv, a.s_local = 0, a.n_split = n_split, a.b_first = 0;
+  a.n_full = -1, a.n_tail = 0, a.tail_parts = 1, a.ws_o = nullptr, a.ws_lse = nullptr;
+  a.scale_log2 = scale_log2, a.rescale_log2 = rescale_log2, a.err = err, a.wait_limit = wait_limit;
+  return launch_any(tq, tk, tv, tq, tk, tv, out, lse, D, a, out_f32, accumulate ? kAccum : kPlain,
+                    stream);
+}
+
+cudaError_t launch_attn_fwd_sm100_tail(const CUtensorMap& tq, const CUtensorMap& tk,
+                                       const CUtensorMap& tv, void* out, float* lse, int B, int H,
+                                       int Sq, int Skv, int D, float scale_log2,
+                                       float rescale_log2, bool out_f32, bool accumulate,
+                                       const TailSplit& t, void* workspace, int* err,
+                                       long long wait_limit, cudaStream_t stream) {
+  const size_t rows = size_t(t.parts) * t.n_tail * (2 * kBlockM);
+  Launch a{};
+  a.grid = dim3(unsigned(t.n_full + t.n_tail * t.parts), 1, 1);
+  a.H = H, a.Sq = Sq, a.Skv = Skv, a.s_local = 0, a.n_split = 1, a.b_first = 0;
+  a.n_full = t.n_full, a.n_tail = t.n_tail, a.tail_parts = t.parts;
+  a.ws_o = static_cast<float*>(workspace);
+  a.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                      ((rows * D * 4 + 255) & ~size_t(255)));
+  a.scale_log2 = scale_log2, a.rescale_log2 = rescale_log2, a.err = err, a.wait_limit = wait_limit;
+  cudaError_t e = launch_any(tq, tk, tv, tq, tk, tv, out, lse, D, a, out_f32,
+                             accumulate ? kAccum : kPlain, stream);
+  if (e != cudaSuccess) return e;
+  return launch_combine_tail(a.ws_o, a.ws_lse, t.n_full, t.n_tail, t.parts, out, lse, B, H, Sq,
+                             D, out_f32 ? 4 : 2, accumulate, stream);
 }
 
 cudaError_t launch_ulysses_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
                                      const CUtensorMap& tv, const CUtensorMap& tq16,
                                      const CUtensorMap& tk16, const CUtensorMap& tv16, void* out,
                                      float* lse, int P, int S_local, int H, int D,
-                                     float scale_log2, float rescale_log2, bool out_f32, int* err,
-                                     long long wait_limit, cudaStream_t stream) {
+                                     float scale_log2, float rescale_log2, bool out_f32,
+                                     int g_first, int n_groups, int* err, long long wait_limit,
+                                     cudaStream_t stream) {
   const int S = P * S_local, Hp = H / P;
-  const long long n_items = (long long)((S + 2 * kBlockM - 1) / (2 * kBlockM)) * Hp * P;
-  if (n_items > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  const Launch a{P, Hp, S, S, S_local, 1, int(n_items), scale_log2, rescale_log2, err,
-                 wait_limit};
+  Launch a{};
+  a.grid = dim3((S + 2 * kBlockM - 1) / (2 * kBlockM), Hp, n_groups);
+  a.H = Hp, a.Sq = S, a.Skv = S, a.s_local = S_local, a.n_split = 1, a.b_first = g_first;
+  a.n_full = -1, a.n_tail = 0, a.tail_parts = 1, a.ws_o = nullptr, a.ws_lse = nullptr;
+  a.scale_log2 = scale_log2, a.rescale_log2 = rescale_log2, a.err = err, a.wait_limit = wait_limit;
   return launch_any(tq, tk, tv, tq16, tk16, tv16, out, lse, D, a, out_f32, kSharded, stream);
 }
 

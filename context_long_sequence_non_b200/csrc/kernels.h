@@ -22,16 +22,43 @@ cudaError_t launch_attn_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
                                   bool out_f32, bool accumulate, int n_split, int* err,
                                   long long wait_limit, cudaStream_t stream);
 
+// Tail split of a single-pass attention launch: the first n_full work items (256-row tile
+// pair x head x batch; whole waves of one CTA per SM) run over all keys, the last n_tail
+// items each as `parts` key ranges whose fp32 partials go to a workspace and are folded by
+// a combine kernel.  parts < 2: nothing to gain, run the plain launch.
+struct TailSplit {
+  int n_full, n_tail, parts;
+};
+TailSplit tail_split_plan(int B, int H, int Sq, int Skv);
+size_t tail_split_workspace(const TailSplit& t, int D);  // bytes (0 when parts < 2)
+
+// The attention (plain or accumulate) with a tail split, then the combine of the tail
+// items' partials into (out, lse) -- with `accumulate`, merged into the running (out, lse).
+cudaError_t launch_attn_fwd_sm100_tail(const CUtensorMap& tq, const CUtensorMap& tk,
+                                       const CUtensorMap& tv, void* out, float* lse, int B, int H,
+                                       int Sq, int Skv, int D, float scale_log2,
+                                       float rescale_log2, bool out_f32, bool accumulate,
+                                       const TailSplit& t, void* workspace, int* err,
+                                       long long wait_limit, cudaStream_t stream);
+
+// Fold the tail items' key-range partials (fp32 O rows [parts][n_tail][256][D], LSE
+// [parts][n_tail][256]) -- and with `accumulate` the running (out, lse) -- into out / lse.
+cudaError_t launch_combine_tail(const float* ws_o, const float* ws_lse, int n_full, int n_tail,
+                                int parts, void* out, float* lse, int B, int H, int Sq, int D,
+                                int out_bytes, bool accumulate, cudaStream_t stream);
+
 // Ulysses fused: q/k/v/out are [P][S_local][H][D] rank shards, each described by two tensor
 // maps over dims (D, H, S_local, P): a 64 x 1 x 128 x 1 box and a 64 x 1 x 16 x 1 box (for
-// tiles that straddle two shards); LSE is [P][H/P][P*S_local].
+// tiles that straddle two shards); LSE is [P][H/P][P*S_local].  The launch computes head
+// groups g_first .. g_first + n_groups - 1 (all P for the whole pass); it reads and writes
+// only those groups' heads.
 cudaError_t launch_ulysses_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
                                      const CUtensorMap& tv, const CUtensorMap& tq16,
                                      const CUtensorMap& tk16, const CUtensorMap& tv16, void* out,
                                      float* lse, int P,
                                      int S_local, int H, int D, float scale_log2,
-                                     float rescale_log2, bool out_f32, int* err,
-                                     long long wait_limit, cudaStream_t stream);
+                                     float rescale_log2, bool out_f32, int g_first, int n_groups,
+                                     int* err, long long wait_limit, cudaStream_t stream);
 
 // Running-max policy of the tensor-core kernel: 0 = exact running max (the dominant key's
 // P is exactly 1, so its bf16 rounding costs nothing).

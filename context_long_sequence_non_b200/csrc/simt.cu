@@ -13,6 +13,35 @@
 namespace cpattn {
 namespace {
 
+// ------------------------------------------------------------------ dependent launches
+// The bandwidth-bound kernels below are launched with programmatic stream serialization: a
+// launch may be scheduled while the previous kernel on the stream is still finishing, and
+// each CTA first waits (griddepcontrol.wait, a hardware dependency) until that kernel has
+// completed and its writes are visible, then lets the next launch be scheduled.  A
+// back-to-back burst (three seq2heads, a ring step's merges) then overlaps each launch's
+// start-up with its predecessor's tail instead of paying it in full.  After a kernel that
+// was not launched this way the wait returns at once and ordering is the stream's.
+__device__ __forceinline__ void dependent_launch_gate() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, cudaStream_t stream,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // ------------------------------------------------------------------ fp32 attention
 // One warp per query row (b, h, i); lane l holds q[d] for d = l, l + 32, ...  Keys are
 // visited in order with an online softmax in fp32 (natural base, expf/logf).
@@ -83,6 +112,7 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(const float* __restrict__
 
 // ------------------------------------------------------------------ empty key set
 __global__ void fill_empty_kernel(uint4* out, size_t n_vec, float* lse, size_t n_lse) {
+  dependent_launch_gate();
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_vec; i += stride)
     out[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -128,6 +158,7 @@ template <bool kBf16>
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
     const uint4* o_a, const float* lse_a, const uint4* o_b, const float* lse_b, uint4* o,
     float* lse, int H, int S, long long n_rows, int vpr) {
+  dependent_launch_gate();
   // a block covers kMergeRowsPerThread groups of (blockDim.x / vpr) consecutive rows; thread
   // (rl, v) takes vector v of row rl of every group, issuing all loads before any math
   const int rows_per_group = blockDim.x / vpr;
@@ -193,6 +224,7 @@ template <bool kBf16>
 __global__ void __launch_bounds__(kMergeThreads, 4) merge_rows_kernel(
     const uint4* o_a, const float* lse_a, const uint4* o_b, const float* lse_b, uint4* o,
     float* lse, int H, int S, int n_vec, int vpr_log2) {
+  dependent_launch_gate();
   const int lane = threadIdx.x & 31;
   const int warp = int((blockIdx.x * kMergeThreads + threadIdx.x) >> 5);
   const int n_warps = int((gridDim.x * kMergeThreads) >> 5);
@@ -259,6 +291,7 @@ __global__ void __launch_bounds__(kMergeThreads) combine_kernel(
     const uint4* __restrict__ part_o, const float* __restrict__ part_lse, int n,
     long long o_stride, long long lse_stride, uint4* out, float* lse, int H, int S,
     long long n_rows, int vpr) {
+  dependent_launch_gate();
   const int rows_per_block = blockDim.x / vpr;
   const int rl = threadIdx.x / vpr;
   const int v = threadIdx.x - rl * vpr;
@@ -323,6 +356,80 @@ __global__ void __launch_bounds__(kMergeThreads) combine_kernel(
   }
   __syncthreads();
   if (live && v == 0 && lse != nullptr) lse[li] = L;
+}
+
+// ------------------------------------------------------------------ tail-split combine
+// The items of the attention launch's last wave were split into `parts` key ranges; range p
+// of tail item t left its normalised fp32 partial (O row, LSE) at workspace row
+// (p * n_tail + t) * 256 + r.  One warp per query row folds them with the n-term merge
+// L = max + ln sum_p exp(L_p - max), O = sum_p exp(L_p - L) O_p -- together with the running
+// (out, lse) row when accumulating (a running LSE of -inf means an empty accumulator whose
+// row is not read) -- and writes the row of out / lse.  Lane l holds D/32 consecutive
+// elements of the row.
+template <int VPL, bool kOutBf16, bool kAcc>
+__global__ void __launch_bounds__(256) combine_tail_kernel(
+    const float* __restrict__ ws_o, const float* __restrict__ ws_lse, int n_full, int n_tail,
+    int parts, void* out, float* lse, int H, int Sq) {
+  dependent_launch_gate();
+  constexpr int D = 32 * VPL;
+  const int lane = threadIdx.x & 31;
+  const int wrow = int(blockIdx.x) * 8 + int(threadIdx.x >> 5);  // tail row (t, r)
+  if (wrow >= n_tail * 256) return;
+  const int t = wrow >> 8, r = wrow & 255;
+  const int n_pairs = (Sq + 255) / 256;
+  const int item = n_full + t;
+  const int pair = item % n_pairs, h = (item / n_pairs) % H, b = item / n_pairs / H;
+  const int q = pair * 256 + r;
+  if (q >= Sq) return;  // rows past the end of the sequence were never written
+  const size_t li = (size_t(b) * H + h) * Sq + q;
+  const size_t orow = ((size_t(b) * Sq + q) * H + h) * D + lane * VPL;
+  float lp[8];
+  float mx = -INFINITY;
+  for (int p = 0; p < parts; ++p) {
+    lp[p] = ws_lse[size_t(p * n_tail + t) * 256 + r];
+    mx = fmaxf(mx, lp[p]);
+  }
+  const float la = kAcc ? lse[li] : -INFINITY;
+  mx = fmaxf(mx, la);
+  float acc[VPL];
+#pragma unroll
+  for (int e = 0; e < VPL; ++e) acc[e] = 0.f;
+  float tot = 0.f;
+  for (int p = 0; p < parts; ++p) {
+    const float w = expf(lp[p] - mx);
+    tot += w;
+    const float* src = ws_o + (size_t(p * n_tail + t) * 256 + r) * D + lane * VPL;
+#pragma unroll
+    for (int e = 0; e < VPL; ++e) acc[e] = fmaf(w, src[e], acc[e]);
+  }
+  if (kAcc && la != -INFINITY) {
+    const float w = expf(la - mx);
+    tot += w;
+    if constexpr (kOutBf16) {
+      const uint16_t* a = static_cast<const uint16_t*>(out) + orow;
+#pragma unroll
+      for (int e = 0; e < VPL; ++e) acc[e] = fmaf(w, __uint_as_float(uint32_t(a[e]) << 16), acc[e]);
+    } else {
+      const float* a = static_cast<const float*>(out) + orow;
+#pragma unroll
+      for (int e = 0; e < VPL; ++e) acc[e] = fmaf(w, a[e], acc[e]);
+    }
+  }
+  const float inv = 1.0f / tot;
+  if constexpr (kOutBf16) {
+    uint32_t w2[VPL / 2];
+#pragma unroll
+    for (int e = 0; e < VPL / 2; ++e) w2[e] = pack_bf16x2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(out) + orow);
+#pragma unroll
+    for (int e = 0; e < VPL / 2; ++e) dst[e] = w2[e];
+  } else {
+    float* dst = static_cast<float*>(out) + orow;
+#pragma unroll
+    for (int e = 0; e < VPL; ++e) dst[e] = acc[e] * inv;
+  }
+  __syncwarp();  // every lane's read of lse[li] precedes lane 0's write
+  if (lane == 0 && lse != nullptr) lse[li] = mx + logf(tot);
 }
 
 // ------------------------------------------------------------------ Ulysses permutes
@@ -414,6 +521,7 @@ __global__ void __launch_bounds__(kPermThreads, 5) permute_kernel(const __grid_c
                                                                 const __grid_constant__ RowNorm nrm,
                                                                 int P, int S_l, int run_vec,
                                                                 int chunks, int n_items) {
+  dependent_launch_gate();
   // blockIdx.y picks the tensor (uniform per block); item = (dst row, 32-vector chunk)
   const int bx = int(blockIdx.x);
   const int tsr = int(bx >= set.block_begin[1]) + int(bx >= set.block_begin[2]);  // tensor
@@ -565,9 +673,8 @@ cudaError_t launch_fill_empty(void* out, size_t out_bytes, float* lse, size_t n_
                               cudaStream_t stream) {
   const size_t n_vec = out_bytes / 16;
   const long long work = (long long)(n_vec > n_lse ? n_vec : n_lse);
-  fill_empty_kernel<<<unsigned(grid_for(work, 256, 8)), 256, 0, stream>>>(
-      static_cast<uint4*>(out), n_vec, lse, n_lse);
-  return cudaGetLastError();
+  return launch_dependent(fill_empty_kernel, dim3(unsigned(grid_for(work, 256, 8))), dim3(256),
+                          stream, static_cast<uint4*>(out), n_vec, lse, n_lse);
 }
 
 cudaError_t launch_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
@@ -584,30 +691,20 @@ cudaError_t launch_merge(const void* o_a, const float* lse_a, const void* o_b, c
     const long long blocks_needed = (warps_needed * 32 + kMergeThreads - 1) / kMergeThreads;
     const long long cap = (long long)sm_count() * 4;  // all resident (64 registers a thread)
     const unsigned blocks = unsigned(blocks_needed < cap ? blocks_needed : cap);
-    if (elem_bytes == 2)
-      merge_rows_kernel<true><<<blocks, kMergeThreads, 0, stream>>>(
-          static_cast<const uint4*>(o_a), lse_a, static_cast<const uint4*>(o_b), lse_b,
-          static_cast<uint4*>(o), lse, H, S, int(n_vec), vpr_log2);
-    else
-      merge_rows_kernel<false><<<blocks, kMergeThreads, 0, stream>>>(
-          static_cast<const uint4*>(o_a), lse_a, static_cast<const uint4*>(o_b), lse_b,
-          static_cast<uint4*>(o), lse, H, S, int(n_vec), vpr_log2);
-    return cudaGetLastError();
+    return launch_dependent(elem_bytes == 2 ? merge_rows_kernel<true> : merge_rows_kernel<false>,
+                            dim3(blocks), dim3(kMergeThreads), stream,
+                            static_cast<const uint4*>(o_a), lse_a, static_cast<const uint4*>(o_b),
+                            lse_b, static_cast<uint4*>(o), lse, H, S, int(n_vec), vpr_log2);
   }
   const int rows_per_group = vpr >= kMergeThreads ? 1 : kMergeThreads / vpr;
   const long long rows_per_block = (long long)rows_per_group * kMergeRowsPerThread;
   const long long blocks = (n_rows + rows_per_block - 1) / rows_per_block;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const int threads = rows_per_group * vpr;
-  if (elem_bytes == 2)
-    merge_kernel<true><<<unsigned(blocks), threads, 0, stream>>>(
-        static_cast<const uint4*>(o_a), lse_a, static_cast<const uint4*>(o_b), lse_b,
-        static_cast<uint4*>(o), lse, H, S, n_rows, vpr);
-  else
-    merge_kernel<false><<<unsigned(blocks), threads, 0, stream>>>(
-        static_cast<const uint4*>(o_a), lse_a, static_cast<const uint4*>(o_b), lse_b,
-        static_cast<uint4*>(o), lse, H, S, n_rows, vpr);
-  return cudaGetLastError();
+  return launch_dependent(elem_bytes == 2 ? merge_kernel<true> : merge_kernel<false>,
+                          dim3(unsigned(blocks)), dim3(threads), stream,
+                          static_cast<const uint4*>(o_a), lse_a, static_cast<const uint4*>(o_b),
+                          lse_b, static_cast<uint4*>(o), lse, H, S, n_rows, vpr);
 }
 
 cudaError_t launch_combine(const void* part_o, const float* part_lse, int n, void* out, float* lse,
@@ -624,19 +721,26 @@ cudaError_t launch_combine(const void* part_o, const float* part_lse, int n, voi
   const long long lse_stride = (long long)B * H * S;
   const uint4* po = static_cast<const uint4*>(part_o);
   uint4* o = static_cast<uint4*>(out);
-#define CPATTN_COMBINE(BF, ACC)                                                             \
-  combine_kernel<BF, ACC><<<unsigned(blocks), threads, 0, stream>>>(po, part_lse, n, o_stride, \
-                                                                    lse_stride, o, lse, H, S,   \
-                                                                    n_rows, vpr)
-  if (elem_bytes == 2) {
-    if (accumulate) CPATTN_COMBINE(true, true);
-    else CPATTN_COMBINE(true, false);
-  } else {
-    if (accumulate) CPATTN_COMBINE(false, true);
-    else CPATTN_COMBINE(false, false);
-  }
-#undef CPATTN_COMBINE
-  return cudaGetLastError();
+  auto kernel = elem_bytes == 2 ? (accumulate ? combine_kernel<true, true> : combine_kernel<true, false>)
+                                : (accumulate ? combine_kernel<false, true> : combine_kernel<false, false>);
+  return launch_dependent(kernel, dim3(unsigned(blocks)), dim3(threads), stream, po, part_lse, n,
+                          o_stride, lse_stride, o, lse, H, S, n_rows, vpr);
+}
+
+cudaError_t launch_combine_tail(const float* ws_o, const float* ws_lse, int n_full, int n_tail,
+                                int parts, void* out, float* lse, int B, int H, int Sq, int D,
+                                int out_bytes, bool accumulate, cudaStream_t stream) {
+  (void)B;
+  if (parts < 1 || parts > 8 || n_tail < 1 || (D != 64 && D != 128)) return cudaErrorInvalidValue;
+  const unsigned blocks = unsigned((n_tail * 256 + 7) / 8);
+  const bool bf = out_bytes == 2;
+  auto kernel = D == 128
+      ? (bf ? (accumulate ? combine_tail_kernel<4, true, true> : combine_tail_kernel<4, true, false>)
+            : (accumulate ? combine_tail_kernel<4, false, true> : combine_tail_kernel<4, false, false>))
+      : (bf ? (accumulate ? combine_tail_kernel<2, true, true> : combine_tail_kernel<2, true, false>)
+            : (accumulate ? combine_tail_kernel<2, false, true> : combine_tail_kernel<2, false, false>));
+  return launch_dependent(kernel, dim3(blocks), dim3(256), stream, ws_o, ws_lse, n_full, n_tail,
+                          parts, out, lse, H, Sq);
 }
 
 static cudaError_t launch_permute(bool to_head, const void* const* src, void* const* dst,
@@ -673,16 +777,11 @@ static cudaError_t launch_permute(bool to_head, const void* const* src, void* co
   }
   const dim3 grid{unsigned(set.block_begin[3]), 1u, 1u};
   const RowNorm none{};
-  if (nrm != nullptr)
-    permute_kernel<true, true><<<grid, kPermThreads, 0, stream>>>(set, *nrm, P, S_local,
-                                                                  int(run_vec), chunks, int(n_items));
-  else if (to_head)
-    permute_kernel<true, false><<<grid, kPermThreads, 0, stream>>>(set, none, P, S_local,
-                                                                   int(run_vec), chunks, int(n_items));
-  else
-    permute_kernel<false, false><<<grid, kPermThreads, 0, stream>>>(set, none, P, S_local,
-                                                                    int(run_vec), chunks, int(n_items));
-  return cudaGetLastError();
+  auto kernel = nrm != nullptr ? permute_kernel<true, true>
+                               : (to_head ? permute_kernel<true, false> : permute_kernel<false, false>);
+  return launch_dependent(kernel, grid, dim3(kPermThreads), stream, set,
+                          nrm != nullptr ? *nrm : none, P, S_local, int(run_vec), chunks,
+                          int(n_items));
 }
 
 static RowNorm row_norm(const float* g0, const float* g1, const float* g2, int D, float eps,
@@ -714,6 +813,7 @@ __global__ void __launch_bounds__(kPermThreads, 5) rmsnorm_kernel(const uint4* _
                                                                   int n_vec, int row_vec,
                                                                   float inv_d, float eps,
                                                                   float out_scale) {
+  dependent_launch_gate();
   const int lane = threadIdx.x & 31;
   const int warp = int((blockIdx.x * kPermThreads + threadIdx.x) >> 5);
   const int n_warps = int((gridDim.x * kPermThreads) >> 5);
@@ -748,10 +848,9 @@ cudaError_t launch_rmsnorm(const void* x, void* y, const float* gamma, long long
   const long long blocks_needed = (warps_needed * 32 + kPermThreads - 1) / kPermThreads;
   const long long cap = (long long)sm_count() * 8;
   const long long blocks = blocks_needed < cap ? blocks_needed : cap;
-  rmsnorm_kernel<<<unsigned(blocks), kPermThreads, 0, stream>>>(
-      static_cast<const uint4*>(x), static_cast<uint4*>(y), gamma, int(n_vec), row_vec,
-      1.0f / float(D), eps, out_scale);
-  return cudaGetLastError();
+  return launch_dependent(rmsnorm_kernel, dim3(unsigned(blocks)), dim3(kPermThreads), stream,
+                          static_cast<const uint4*>(x), static_cast<uint4*>(y), gamma, int(n_vec),
+                          row_vec, 1.0f / float(D), eps, out_scale);
 }
 
 cudaError_t launch_seq2head(const void* src, void* dst, int P, int S_local, long long run_vec,

@@ -121,6 +121,23 @@ __device__ __forceinline__ bool bar_and(uint32_t id, uint32_t count, bool ok) {
   return r != 0;
 }
 
+// ------------------------------------------------------------------ dependent launches
+
+// Wait until the kernel that precedes this grid on its stream has completed and its memory
+// writes are visible (returns at once when this grid was not launched as a dependent).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Allow the next kernel on the stream, if launched as a dependent, to be scheduled now (it
+// still waits for this grid's completion before touching memory).
+__device__ __forceinline__ void griddep_release() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Fetch the 128-byte line holding `p` into L2 ahead of its use.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

@@ -29,7 +29,8 @@ def ring_attention(q, k_chunks, v_chunks, scale=None, acc_dtype=None, fused=True
     writes each chunk's partial and folds it with the separate merge kernel.  With the fused
     form, ``n_split`` > 1 (or None: the library's suggestion) computes every chunk as that
     many key ranges folded straight into the accumulator (split-KV, for query slices too
-    small to fill the GPU).  Returns ``(O, LSE)``.
+    small to fill the GPU), and ``n_split = 0`` splits only the work items of each chunk's
+    last, partial wave of CTAs (tail split).  Returns ``(O, LSE)``.
     """
     if scale is None:
         scale = 1.0 / math.sqrt(q.shape[3])
@@ -40,7 +41,7 @@ def ring_attention(q, k_chunks, v_chunks, scale=None, acc_dtype=None, fused=True
     if fused:
         if n_split is None:
             n_split = B.split_suggest(Bn, H, Sq, k_chunks[0].shape[1])
-        if n_split > 1:
+        if n_split != 1:
             ws = torch.empty(max(B.split_workspace_bytes(Bn, H, Sq, D, n_split, acc_dtype), 256),
                              dtype=torch.uint8, device=q.device)
             acc_l.fill_(-math.inf)  # empty accumulator: its O rows are never read
@@ -168,3 +169,27 @@ class UlyssesStreamer:
             self.downloaded[k].record(self.download)
         self.step += 1
         return self.downloaded[k]
+
+
+class UlyssesHostPass:
+    """A whole Ulysses attention layer from host memory to host memory in one C-ABI call
+    (cpattn_ulysses_host).  The device work buffers are allocated here once, by PyTorch;
+    the library allocates nothing.  Inside the call the head groups go in ``n_chunks``
+    chunks: the upload of chunk c+1 and the download of chunk c-1 overlap the attention of
+    chunk c.  Host tensors should be pinned."""
+
+    def __init__(self, P, S_local, H, D, out_dtype=torch.bfloat16, device="cuda", n_chunks=None,
+                 with_lse=True):
+        shard = (P, S_local, H, D)
+        self.P, self.n_chunks = P, n_chunks if n_chunks is not None else max(1, P // 2)
+        self.dq, self.dk, self.dv = (torch.empty(shard, dtype=torch.bfloat16, device=device)
+                                     for _ in range(3))
+        self.d_out = torch.empty(shard, dtype=out_dtype, device=device)
+        self.d_lse = (torch.empty((P, H // P, P * S_local), dtype=torch.float32, device=device)
+                      if with_lse else None)
+
+    def run(self, hq, hk, hv, h_out, h_lse=None, scale=None, stream=None):
+        """Enqueue one pass; h_out / h_lse are valid once ``stream`` has passed it."""
+        return B.ulysses_host(hq, hk, hv, h_out, h_lse, self.dq, self.dk, self.dv, self.d_out,
+                              self.d_lse if h_lse is not None else None, self.P, scale=scale,
+                              n_chunks=self.n_chunks, stream=stream)

@@ -172,6 +172,41 @@ CPATTN_API int cpattn_ulysses_fwd(const void* q, const void* k, const void* v, v
                                   int out_dtype, cpattn_stream_t stream);
 
 /*
+ * cpattn_ulysses_host -- cpattn_ulysses_fwd from host memory to host memory: one whole
+ * Ulysses attention layer (Fig. 4) whose Q/K/V rank shards are in host memory and whose O
+ * and LSE are wanted back in host memory, as in a host-driven inference loop (warm-up,
+ * then timed iterations: the attention_mdtrt guide, section 推理程序运行机制).  The head
+ * groups are processed in n_chunks chunks (chunk c = groups [c*P/n_chunks,
+ * (c+1)*P/n_chunks)), pipelined so that the copies overlap the attention:
+ *   upload stream:   Q, K, V heads of chunk c  host -> device  (one 2-D copy per tensor)
+ *   compute streams: attention of chunk c      (the fused Ulysses kernel, chunk c only;
+ *                    neighbouring chunks on two streams, so one chunk's last wave of work
+ *                    overlaps the next chunk's first)
+ *   download stream: O heads and LSE rows of chunk c  device -> host
+ * ordered by events.  The result equals cpattn_ulysses_fwd on the same shards bit for bit.
+ * h_q, h_k, h_v : [P][S_local][H][D] bf16 in host memory (page-locked, or the copies are
+ *   not asynchronous); h_out : [P][S_local][H][D] out_dtype; h_lse : [P][H/P][P*S_local]
+ *   float32, or NULL (then d_lse must be NULL too).
+ * d_q, d_k, d_v, d_out, d_lse : caller-owned device buffers of the same shapes (the call
+ *   allocates nothing), pairwise disjoint.
+ * All work is ordered after the work already on `stream`, and `stream` waits for all of it
+ * (the last copy to the host) before anything enqueued on it later; the call returns once
+ * everything is enqueued.  Host outputs may be read, and host inputs reused, only after
+ * `stream` has reached that point (cudaStreamSynchronize, or an event recorded on it).
+ * The upload, download and second compute streams and four events per device are created
+ * on the first call on that device and kept until the process exits; calls on one device
+ * from several threads are enqueued one at a time.
+ * n_chunks in 1..P (P/2 chunks of two groups each is a good default at P = 8); other
+ * requirements and errors as cpattn_ulysses_fwd, plus CPATTN_ERR_SHAPE for n_chunks or
+ * overlapping device buffers and CPATTN_ERR_NULL for a missing host pointer.
+ */
+CPATTN_API int cpattn_ulysses_host(const void* h_q, const void* h_k, const void* h_v,
+                                   void* h_out, float* h_lse, void* d_q, void* d_k, void* d_v,
+                                   void* d_out, float* d_lse, int P, int S_local, int H, int D,
+                                   float scale, int out_dtype, int n_chunks,
+                                   cpattn_stream_t stream);
+
+/*
  * cpattn_fwd_accumulate -- one Ring Attention step with the merge fused into the attention
  * epilogue (环形注意力 / Ring Attention, Fig. 3: each rank folds every arriving K/V chunk
  * into its running result with the online softmax).  Computes the chunk's partial

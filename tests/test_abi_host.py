@@ -101,6 +101,30 @@ def test_ulysses_fwd_argument_errors(L):
     assert uf(q=FAKE + 8) == B.ERR_ALIGN
 
 
+def test_ulysses_host_argument_errors(L):
+    vp = ctypes.c_void_p
+    H0, D0 = 0x7000000, 0x100000000  # fake host and device addresses (never dereferenced)
+    step = 0x10000000
+
+    def uh(P=2, S_l=32, H=4, D=128, n=1, hq=H0, hl=H0 + 5 * step, dl=D0 + 4 * step, dq=D0,
+           dk=D0 + step, dout=0):
+        return L.cpattn_ulysses_host(vp(hq) if hq else None, vp(H0 + step), vp(H0 + 2 * step),
+                                     vp(H0 + 3 * step), vp(hl) if hl else None,
+                                     vp(dq) if dq else None, vp(dk), vp(D0 + 2 * step),
+                                     vp(D0 + 3 * step), vp(dl) if dl else None, P, S_l, H, D,
+                                     0.1, dout, n, None)
+
+    assert uh(H=5) == B.ERR_SHAPE
+    assert uh(S_l=24) == B.ERR_UNSUPPORTED
+    assert uh(n=0) == B.ERR_SHAPE and uh(n=3) == B.ERR_SHAPE  # chunks in 1..P
+    assert uh(hq=0) == B.ERR_NULL
+    assert uh(dq=0) == B.ERR_NULL
+    assert uh(hl=0) == B.ERR_NULL  # h_lse and d_lse go together
+    assert uh(dq=D0 + 8) == B.ERR_ALIGN
+    assert uh(dk=D0 + 64) == B.ERR_SHAPE  # device buffers overlap
+    assert uh(dout=5) == B.ERR_UNSUPPORTED
+
+
 def test_fwd_split_argument_errors_and_sizes(L):
     vp = ctypes.c_void_p
 
@@ -110,7 +134,9 @@ def test_fwd_split_argument_errors_and_sizes(L):
                                   ws_bytes, None)
 
     assert fs(n=9) == B.ERR_SHAPE
-    assert fs(n=0) == B.ERR_SHAPE
+    assert fs(n=-1) == B.ERR_SHAPE
+    assert fs(n=0, ws_bytes=1000) == B.ERR_SHAPE  # tail split: 4 items split 8 ways
+    assert fs(n=0, ws=0) == B.ERR_NULL
     assert fs(ws=0) == B.ERR_NULL
     assert fs(ws=FAKE + 16) == B.ERR_ALIGN  # 256-byte alignment
     assert fs(ws_bytes=1000) == B.ERR_SHAPE  # too small
@@ -120,16 +146,18 @@ def test_fwd_split_argument_errors_and_sizes(L):
     assert need == 2 * 512 * 2 * 128 * 2 + 2 * 2 * 512 * 4
     assert L.cpattn_fwd_split_workspace(1, 2, 512, 128, 1, 0) == 0
     assert L.cpattn_fwd_split_workspace(1, 2, 512, 128, 9, 0) == 0
+    # n_split = 0 (tail split) on 148 SMs: 352 items of a [5520][16][128] query leave 56 in
+    # the last wave, each split in 2: fp32 rows of 2 * 56 * 256, then their LSEs
+    rows = 2 * 56 * 256
+    assert L.cpattn_fwd_split_workspace(1, 16, 5520, 128, 0, 0) == rows * 128 * 4 + rows * 4
+    assert L.cpattn_fwd_split_workspace(8, 2, 44160, 128, 0, 0) == 0  # 104 left: no room to split
+    assert L.cpattn_fwd_split_workspace(1, 16, 5520, 96, 0, 0) == 0
 
 
 def test_split_suggestion_model():
-    # work items are (256-row tile pair, head, key range) on 148 persistent CTAs (no GPU
-    # here: the library's default SM count)
-    assert B.split_suggest(8, 2, 44160, 44160) == 1  # 2768 items: 18.7 rounds already
-    assert B.split_suggest(1, 24, 4608, 4608) == 1   # 432 items: 2.92 rounds, nothing to gain
-    assert B.split_suggest(1, 16, 512, 44160) == 4   # 32 items over 345 key blocks: split
-    # 352 items of 43 blocks = 2.38 rounds; two ranges give 704 half items = 4.76 rounds
-    assert B.split_suggest(1, 16, 5520, 5520) == 2
+    assert B.split_suggest(8, 2, 44160, 44160) == 1  # 2768 CTAs: many waves already
+    assert B.split_suggest(1, 16, 512, 44160) >= 4   # 32 CTAs over 345 key blocks: split
+    assert B.split_suggest(1, 16, 5520, 5520) == 1   # 352 CTAs of 43 blocks: start-up eats it
     assert B.split_suggest(1, 1, 128, 128) == 1       # too few key blocks to split
 
 

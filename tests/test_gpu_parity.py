@@ -305,6 +305,55 @@ def test_split_kv_matches_single_pass_and_oracle(shape, n_split, out_dtype):
     assert (o_a.float() - o_s.float()).abs().max().item() < tol
 
 
+# Tail split (n_split = 0): the work items of the last, partial wave of CTAs are computed as
+# key ranges whose fp32 partials a combine kernel folds; every other item is computed whole.
+@pytest.mark.parametrize("shape", [(1, 3, 300, 1000, 128), (2, 5, 700, 517, 64),
+                                   (1, 37, 1100, 900, 128)])  # 185 items: 37 in the tail
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_tail_split_matches_oracle(shape, out_dtype):
+    Bn, H, Sq, Skv, D = shape
+    q, k, v = W.random_case(Sq + Skv + H, Bn, H, Sq, Skv, D)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    need = cp.split_workspace_bytes(Bn, H, Sq, D, 0, out_dtype)
+    assert need > 0
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device=DEV)  # garbage in the workspace
+    o_t, l_t = cp.fwd_split(qd, kd, vd, out_dtype=out_dtype, n_split=0, workspace=ws)
+    o_1, l_1 = cp.fwd(qd, kd, vd, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    o_ref, l_ref = ref.attention(q, k, v, 1 / math.sqrt(D))
+    kind = "bf16_out" if out_dtype == torch.bfloat16 else "bf16_in"
+    check_o(o_t, o_ref, kind, f"tail split {shape}")
+    check_lse(l_t, l_ref, f"tail split {shape}")
+    assert (l_t - l_1).abs().max().item() < 2e-5
+    # accumulate: a second pass over the same keys adds ln 2 and keeps O
+    o_a, l_a = o_t.clone(), l_t.clone()
+    cp.fwd_split(qd, kd, vd, out=o_a, lse=l_a, accumulate=True, n_split=0, workspace=ws)
+    torch.cuda.synchronize()
+    assert ((l_a - l_t) - math.log(2)).abs().max().item() < 2e-5
+    tol = 2e-5 if out_dtype == torch.float32 else 1e-2
+    assert (o_a.float() - o_t.float()).abs().max().item() < tol
+
+
+def test_ring_step_with_tail_split():
+    # one rank's ring step: 352 items on 148 SMs leave 56 in the last wave, split in two
+    w = W.WORKLOADS[3]
+    x = W.make_inputs(w)
+    q, k, v = (x[n].to(DEV) for n in ("q", "k", "v"))
+    c = x["chunks"][0]
+    kc = [k[:, i * c:(i + 1) * c].contiguous() for i in range(len(x["chunks"]))]
+    vc = [v[:, i * c:(i + 1) * c].contiguous() for i in range(len(x["chunks"]))]
+    o_t, l_t = cp.ring_attention(q, kc, vc, acc_dtype=torch.float32, n_split=0)
+    o_1, l_1 = cp.ring_attention(q, kc, vc, acc_dtype=torch.float32, n_split=1)
+    o_b, l_b = cp.ring_attention(q, kc, vc, n_split=0)  # bf16 accumulator
+    torch.cuda.synchronize()
+    assert (o_t - o_1).abs().max().item() < 2e-3 and (l_t - l_1).abs().max().item() < 2e-5
+    rows = W.sample_rows(w.B, w.H, w.Sq, 1024, seed=34)
+    _sampled(x["q"], x["k"], x["v"], w.softmax_scale, o_t.cpu(), l_t.cpu(), rows, "bf16_in",
+             "ring tail split")
+    _sampled(x["q"], x["k"], x["v"], w.softmax_scale, o_b.cpu(), l_b.cpu(), rows, "bf16_out",
+             "ring tail split bf16")
+
+
 def test_ring_step_with_split_kv():
     w = W.WORKLOADS[3]
     x = W.make_inputs(w)
@@ -425,6 +474,51 @@ def test_fused_ulysses_full_size_bit_identical():
     out_u, lse_u = plan.run(q, k, v)
     torch.cuda.synchronize()
     assert torch.equal(out_f, out_u) and torch.equal(lse_f, lse_u)
+
+
+# ----------------------------------------------------------------------------- host-buffer pass
+
+
+@pytest.mark.parametrize("n_chunks", [1, 2, 3, 4])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_ulysses_host_pass_equals_device_path(n_chunks, out_dtype):
+    # host shards in, host O/LSE out, copies pipelined over head-group chunks inside the
+    # C-ABI call: the same bits as the device-resident fused call, and the oracle's values
+    P, S_l, H, D = 4, 400, 8, 128
+    g = torch.Generator().manual_seed(900 + n_chunks)
+    host = [W.randn((P, S_l, H, D), g, 1.0, "bf16").pin_memory() for _ in range(3)]
+    h_out = torch.full((P, S_l, H, D), float("nan"), dtype=out_dtype).pin_memory()
+    h_lse = torch.full((P, H // P, P * S_l), float("nan")).pin_memory()
+    hp = cp.UlyssesHostPass(P, S_l, H, D, out_dtype=out_dtype, device=DEV, n_chunks=n_chunks)
+    hp.run(*host, h_out, h_lse)
+    torch.cuda.synchronize()
+    o_d, l_d = cp.ulysses_fwd(*(t.to(DEV) for t in host), P, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert torch.equal(h_out, o_d.cpu()) and torch.equal(h_lse, l_d.cpu())
+    full = lambda t: t.reshape(1, P * S_l, H, D)
+    rows = W.sample_rows(1, H, P * S_l, 512, seed=9)
+    o_ref, l_ref = ref.attention_rows(full(host[0]), full(host[1]), full(host[2]),
+                                      1 / math.sqrt(D), rows)
+    oc, lc = full(h_out), h_lse.reshape(1, H, P * S_l)
+    kind = "bf16_out" if out_dtype == torch.bfloat16 else "bf16_in"
+    check_o(torch.stack([oc[b, i, h] for (b, h, i) in rows]), o_ref, kind, "host pass")
+    check_lse(torch.stack([lc[b, h, i] for (b, h, i) in rows]), l_ref, "host pass")
+
+
+def test_ulysses_host_pass_full_size():
+    w = W.WORKLOADS[4]
+    x = W.make_inputs(w)
+    P, S_l, H = w.P, w.Sq // w.P, w.H * w.P
+    host = [x[n].pin_memory() for n in ("q", "k", "v")]
+    h_out = torch.empty((P, S_l, H, w.D), dtype=torch.bfloat16).pin_memory()
+    h_lse = torch.empty((P, H // P, P * S_l)).pin_memory()
+    hp = cp.UlyssesHostPass(P, S_l, H, w.D, device=DEV)
+    for _ in range(2):  # twice in a row on the same buffers
+        hp.run(*host, h_out, h_lse, scale=w.softmax_scale)
+    torch.cuda.synchronize()
+    o_d, l_d = cp.ulysses_fwd(*(t.to(DEV) for t in host), P, scale=w.softmax_scale)
+    torch.cuda.synchronize()
+    assert torch.equal(h_out, o_d.cpu()) and torch.equal(h_lse, l_d.cpu())
 
 
 # ----------------------------------------------------------------------------- the five workloads
