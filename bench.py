@@ -46,9 +46,9 @@ WORKLOAD = W.WORKLOADS[4]
 ATTN_SOURCES = ("context_long_sequence_non_b200/csrc/attn_sm100.cu",
                 "context_long_sequence_non_b200/csrc/sm100_ptx.cuh")
 ATTN_TRAFFIC = {
-    "attn_fwd_sm100_kernel<128,0,0>": {
-        "sources_sha256": "670a6a10557d5e93274985aea76ef3e33e3c4bdecf726c251274211068314865",
-        "bytes": 597_763_840 + 168_522_496,
+    "attn_fwd_sm100_kernel<128,0,2>": {  # the fused Ulysses kernel, one launch per step
+        "sources_sha256": "c844a105f220fe828b9fdb2708e84001093f60675f95f1175151a0dc3dd457e9",
+        "bytes": 574_993_152 + 168_184_064,
     },
 }
 L2_NOTE = ("inputs larger than L2: each step streams 543 MB of Q/K/V shards plus 724 MB of "
@@ -630,7 +630,7 @@ def e2e_run(cp, UlyssesPlan, w, x, dev, stream, args):
     return {"value": tf(ms_host), "unit": UNIT, "ms_per_step": round(ms_host, 4),
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
             "mode": ("C ABI cpattn_ulysses_host (UlyssesHostPass): pinned host Q/K/V shards in, "
-                     "host O + LSE out; head groups in 4 chunks, uploads and downloads "
+                     "host O + LSE out; one chunk per head group (8), uploads and downloads "
                      "overlapping the attention inside each call; calls back to back"),
             "streamer": {"value": tf(ms_streamer), "ms_per_step": round(ms_streamer, 4),
                          "mode": "UlyssesStreamer: neighbouring steps' copies overlap compute "

@@ -182,7 +182,7 @@ def ulysses_host(hq, hk, hv, h_out, h_lse, dq, dk, dv, d_out, d_lse, P, scale=No
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if n_chunks is None:
-        n_chunks = max(1, P // 2)
+        n_chunks = P
     st = lib().cpattn_ulysses_host(_ptr(hq), _ptr(hk), _ptr(hv), _ptr(h_out), _ptr(h_lse),
                                    _ptr(dq), _ptr(dk), _ptr(dv), _ptr(d_out), _ptr(d_lse), P,
                                    S_l, H, D, float(scale), _dtype_code(d_out.dtype),

@@ -181,7 +181,7 @@ class UlyssesHostPass:
     def __init__(self, P, S_local, H, D, out_dtype=torch.bfloat16, device="cuda", n_chunks=None,
                  with_lse=True):
         shard = (P, S_local, H, D)
-        self.P, self.n_chunks = P, n_chunks if n_chunks is not None else max(1, P // 2)
+        self.P, self.n_chunks = P, n_chunks if n_chunks is not None else P
         self.dq, self.dk, self.dv = (torch.empty(shard, dtype=torch.bfloat16, device=device)
                                      for _ in range(3))
         self.d_out = torch.empty(shard, dtype=out_dtype, device=device)

@@ -196,7 +196,7 @@ CPATTN_API int cpattn_ulysses_fwd(const void* q, const void* k, const void* v, v
  * The upload, download and second compute streams and four events per device are created
  * on the first call on that device and kept until the process exits; calls on one device
  * from several threads are enqueued one at a time.
- * n_chunks in 1..P (P/2 chunks of two groups each is a good default at P = 8); other
+ * n_chunks in 1..P (one chunk per head group, n_chunks = P, was fastest at P = 8); other
  * requirements and errors as cpattn_ulysses_fwd, plus CPATTN_ERR_SHAPE for n_chunks or
  * overlapping device buffers and CPATTN_ERR_NULL for a missing host pointer.
  */
