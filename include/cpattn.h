@@ -55,7 +55,7 @@ typedef enum {
   CPATTN_ERR_NULL = 1,        /* a required pointer is NULL */
   CPATTN_ERR_SHAPE = 2,       /* a size is out of range or inconsistent */
   CPATTN_ERR_ALIGN = 3,       /* a pointer is not suitably aligned */
-  CPATTN_ERR_UNSUPPORTED = 4, /* valid request this build has no kernel for */
+  CPATTN_ERR_UNSUPPORTED = 4, /* valid request the library has no kernel for */
   CPATTN_ERR_CUDA = 5,        /* a CUDA runtime/driver call or launch failed */
   CPATTN_ERR_DEVICE_TIMEOUT = 6 /* a kernel's bounded wait ran out (device error word) */
 } cpattn_status;
