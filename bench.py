@@ -47,8 +47,8 @@ ATTN_SOURCES = ("context_long_sequence_non_b200/csrc/attn_sm100.cu",
                 "context_long_sequence_non_b200/csrc/sm100_ptx.cuh")
 ATTN_TRAFFIC = {
     "attn_fwd_sm100_kernel<128,0,2>": {  # the fused Ulysses kernel, one launch per step
-        "sources_sha256": "c844a105f220fe828b9fdb2708e84001093f60675f95f1175151a0dc3dd457e9",
-        "bytes": 574_993_152 + 168_184_064,
+        "sources_sha256": "cc22e897df40d9a9c09c6b9ba50ff18a9d41e189c17771a08374b346356edc3d",
+        "bytes": 594_595_584 + 169_908_224,
     },
 }
 AUX_REPS = 15  # bursts per auxiliary measurement (median reported, with the range)

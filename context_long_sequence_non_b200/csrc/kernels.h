@@ -60,9 +60,10 @@ cudaError_t launch_ulysses_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& t
                                      float rescale_log2, bool out_f32, int g_first, int n_groups,
                                      int* err, long long wait_limit, cudaStream_t stream);
 
-// Running-max policy of the tensor-core kernel: 0 = exact running max (the dominant key's
-// P is exactly 1, so its bf16 rounding costs nothing).
-constexpr float kRescaleLog2 = 0.0f;
+// Running-max policy of the tensor-core kernel: the reference max of a row moves (and O is
+// rescaled) when a block's max exceeds it by more than this (log2 units), or when a key
+// above it could weigh 1/8 or more of the row's result (see attn_sm100.cu).
+constexpr float kRescaleLog2 = 8.0f;
 
 // fp32 CUDA-core attention, D <= 256.
 cudaError_t launch_attn_fwd_f32(const float* q, const float* k, const float* v, void* out,

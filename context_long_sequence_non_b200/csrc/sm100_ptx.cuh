@@ -473,7 +473,8 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
   return d;
 }
 
-// 2^t for a pair of t <= 0 on the FMA pipe instead of the special-function unit.
+// 2^t for a pair of t <= 8 (the softmax's exponents: at most the 2^8 headroom of its
+// reference max) on the FMA pipe instead of the special-function unit.
 // Cody-Waite: t = n + f with n = round(t) (the 1.5*2^23 shifter), f in [-1/2, 1/2];
 // 2^f ~= 1 + f(c1 + f(c2 + f c3)) with c1..c3 from gen_exp2_poly.py (own constrained
 // minimax fit, constant term exactly 1, max relative error 1.02e-4 in fp32); 2^n is added

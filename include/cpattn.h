@@ -348,7 +348,7 @@ CPATTN_API int cpattn_selftest_wait_timeout(long long limit_cycles, cpattn_strea
  * cpattn_selftest_exp2 -- evaluates, on the device, the polynomial 2^t the attention
  * kernel uses for a fixed share of its softmax exponentials (Cody-Waite range reduction
  * t = n + f, |f| <= 1/2, then a degree-3 polynomial with constant term exactly 1, fitted
- * by csrc/gen_exp2_poly.py; relative error <= 1.02e-4 for -125 <= t <= 0; t below -125
+ * by csrc/gen_exp2_poly.py; relative error <= 1.02e-4 for -125 <= t <= 8; t below -125
  * returns 2^-125).  t, out: n device floats.  For tests against the error bound.
  * Errors: CPATTN_ERR_SHAPE (n < 1), _NULL, _ALIGN, _CUDA.
  */
