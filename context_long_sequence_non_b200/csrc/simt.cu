@@ -480,16 +480,19 @@ __device__ __forceinline__ void load_gamma8(const float* __restrict__ gamma, int
   g[4] = g1.x; g[5] = g1.y; g[6] = g1.z; g[7] = g1.w;
 }
 
-// Normalise the 8 elements of one 16-byte vector; every lane of the warp must call it
-// (dead lanes with live = false contribute nothing and get `in` back).
-__device__ __forceinline__ uint4 rms_normalise(uint4 in, bool live, int row_vec, float inv_d,
-                                               float eps, float out_scale, const float (&g)[8]) {
+// Normalise the 8 elements of one 16-byte vector; every lane of the warp must call it.  A
+// head row (kRowVec lanes) is always either wholly live or wholly dead -- items are
+// warp-uniform and runs are whole head rows -- so a dead lane (whose input is zero, never
+// stored) never mixes into a live row's sum.
+template <int kRowVec>
+__device__ __forceinline__ uint4 rms_normalise(uint4 in, float inv_d, float eps,
+                                               float out_scale, const float (&g)[8]) {
   const uint32_t w[4] = {in.x, in.y, in.z, in.w};
   float f[8];
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
-    f[2 * t] = live ? __uint_as_float(w[t] << 16) : 0.f;  // bf16 -> fp32 is exact
-    f[2 * t + 1] = live ? __uint_as_float(w[t] & 0xFFFF0000u) : 0.f;
+    f[2 * t] = __uint_as_float(w[t] << 16);  // bf16 -> fp32 is exact
+    f[2 * t + 1] = __uint_as_float(w[t] & 0xFFFF0000u);
   }
   // packed fp32x2 arithmetic: per lane the same IEEE operations as the scalar forms, in
   // half the issue slots (the fused permute is issue-bound)
@@ -500,10 +503,10 @@ __device__ __forceinline__ uint4 rms_normalise(uint4 in, bool live, int row_vec,
     ss2 = ffma2(fe, fe, ss2);
   }
   float ss = ss2.x + ss2.y;
-  for (int o = 1; o < row_vec; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+#pragma unroll
+  for (int o = 1; o < kRowVec; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   const float a = ss * inv_d + eps;
   const float r = a > 0.f ? rsqrt_refined(a) : 0.f;  // an all-zero row with eps = 0 stays 0
-  if (!live) return in;
   const float2 r2 = make_float2(r, r), s2 = make_float2(out_scale, out_scale);
   uint32_t w_out[4];
 #pragma unroll
@@ -516,8 +519,10 @@ __device__ __forceinline__ uint4 rms_normalise(uint4 in, bool live, int row_vec,
   return make_uint4(w_out[0], w_out[1], w_out[2], w_out[3]);
 }
 
-template <bool kToHead, bool kNorm>
-__global__ void __launch_bounds__(kPermThreads, 5) permute_kernel(const __grid_constant__ PermuteSet set,
+// kRowVec: 16-byte vectors per head row for the normalising form (D / 8), 0 for a copy.
+// The normalising form takes 4 blocks per SM (its registers without spilling), the copy 5.
+template <bool kToHead, bool kNorm, int kRowVec>
+__global__ void __launch_bounds__(kPermThreads, kNorm ? 4 : 5) permute_kernel(const __grid_constant__ PermuteSet set,
                                                                 const __grid_constant__ RowNorm nrm,
                                                                 int P, int S_l, int run_vec,
                                                                 int chunks, int n_items) {
@@ -564,6 +569,7 @@ __global__ void __launch_bounds__(kPermThreads, 5) permute_kernel(const __grid_c
       const int src_row = kToHead ? (d1 * S_l + d0) * P + d2   // Bq(g, r, s)
                                   : (d0 * P + d2) * S_l + d1;  // A(g, r, s)
       dst_off[u] = (long long)n * run_vec + v;
+      if constexpr (kNorm) buf[u] = make_uint4(0u, 0u, 0u, 0u);
       if (live[u]) buf[u] = src[(long long)src_row * run_vec + v];
       if (++c == chunks) {  // next item: next chunk, else the next dst row
         c = 0;
@@ -581,7 +587,7 @@ __global__ void __launch_bounds__(kPermThreads, 5) permute_kernel(const __grid_c
       if (gamma != nullptr) {
 #pragma unroll
         for (int u = 0; u < kPermUnroll; ++u)
-          buf[u] = rms_normalise(buf[u], live[u], nrm.row_vec, nrm.inv_d, nrm.eps, nrm.out_scale, g);
+          buf[u] = rms_normalise<kRowVec>(buf[u], nrm.inv_d, nrm.eps, nrm.out_scale, g);
       }
     }
 #pragma unroll
@@ -777,8 +783,18 @@ static cudaError_t launch_permute(bool to_head, const void* const* src, void* co
   }
   const dim3 grid{unsigned(set.block_begin[3]), 1u, 1u};
   const RowNorm none{};
-  auto kernel = nrm != nullptr ? permute_kernel<true, true>
-                               : (to_head ? permute_kernel<true, false> : permute_kernel<false, false>);
+  auto kernel = to_head ? permute_kernel<true, false, 0> : permute_kernel<false, false, 0>;
+  if (nrm != nullptr) {
+    switch (nrm->row_vec) {  // D / 8 for D a power of two in [8, 256]
+      case 1: kernel = permute_kernel<true, true, 1>; break;
+      case 2: kernel = permute_kernel<true, true, 2>; break;
+      case 4: kernel = permute_kernel<true, true, 4>; break;
+      case 8: kernel = permute_kernel<true, true, 8>; break;
+      case 16: kernel = permute_kernel<true, true, 16>; break;
+      case 32: kernel = permute_kernel<true, true, 32>; break;
+      default: return cudaErrorInvalidValue;
+    }
+  }
   return launch_dependent(kernel, grid, dim3(kPermThreads), stream, set,
                           nrm != nullptr ? *nrm : none, P, S_local, int(run_vec), chunks,
                           int(n_items));
@@ -807,6 +823,7 @@ cudaError_t launch_seq2head_qkv_norm(const void* const* src, void* const* dst, c
 
 // Standalone RMSNorm over a flat [rows][D] array: item = 32 consecutive vectors (32/row_vec
 // whole head rows), kPermUnroll items per warp in flight; same arithmetic as the fused form.
+template <int kRowVec>
 __global__ void __launch_bounds__(kPermThreads, 5) rmsnorm_kernel(const uint4* __restrict__ x,
                                                                   uint4* __restrict__ y,
                                                                   const float* __restrict__ gamma,
@@ -827,11 +844,12 @@ __global__ void __launch_bounds__(kPermThreads, 5) rmsnorm_kernel(const uint4* _
     for (int u = 0; u < kPermUnroll; ++u) {
       const int v = ((it0 + u) << 5) + lane;  // < 2^31: n_vec + 31 + 32 * kPermUnroll fits
       live[u] = it0 + u < n_items && v < n_vec;
+      buf[u] = make_uint4(0u, 0u, 0u, 0u);
       if (live[u]) buf[u] = x[v];
     }
 #pragma unroll
     for (int u = 0; u < kPermUnroll; ++u)
-      buf[u] = rms_normalise(buf[u], live[u], row_vec, inv_d, eps, out_scale, g);
+      buf[u] = rms_normalise<kRowVec>(buf[u], inv_d, eps, out_scale, g);
 #pragma unroll
     for (int u = 0; u < kPermUnroll; ++u)
       if (live[u]) y[((it0 + u) << 5) + lane] = buf[u];
@@ -848,7 +866,17 @@ cudaError_t launch_rmsnorm(const void* x, void* y, const float* gamma, long long
   const long long blocks_needed = (warps_needed * 32 + kPermThreads - 1) / kPermThreads;
   const long long cap = (long long)sm_count() * 8;
   const long long blocks = blocks_needed < cap ? blocks_needed : cap;
-  return launch_dependent(rmsnorm_kernel, dim3(unsigned(blocks)), dim3(kPermThreads), stream,
+  void (*kernel)(const uint4*, uint4*, const float*, int, int, float, float, float) = nullptr;
+  switch (row_vec) {  // D / 8 for D a power of two in [8, 256]
+    case 1: kernel = rmsnorm_kernel<1>; break;
+    case 2: kernel = rmsnorm_kernel<2>; break;
+    case 4: kernel = rmsnorm_kernel<4>; break;
+    case 8: kernel = rmsnorm_kernel<8>; break;
+    case 16: kernel = rmsnorm_kernel<16>; break;
+    case 32: kernel = rmsnorm_kernel<32>; break;
+    default: return cudaErrorInvalidValue;
+  }
+  return launch_dependent(kernel, dim3(unsigned(blocks)), dim3(kPermThreads), stream,
                           static_cast<const uint4*>(x), static_cast<uint4*>(y), gamma, int(n_vec),
                           row_vec, 1.0f / float(D), eps, out_scale);
 }
