@@ -505,6 +505,27 @@ def test_ulysses_host_pass_equals_device_path(n_chunks, out_dtype):
     check_lse(torch.stack([lc[b, h, i] for (b, h, i) in rows]), l_ref, "host pass")
 
 
+def test_ulysses_host_pass_double_buffered_on_two_streams():
+    # a serving loop: two passes (two device buffer sets) alternate on two streams, so
+    # calls overlap on the GPU and share the library's upload / compute / download streams;
+    # every step's host outputs must still equal the device path on that step's inputs
+    P, S_l, H, D, steps = 4, 272, 8, 128, 6
+    g = torch.Generator().manual_seed(505)
+    host = [[W.randn((P, S_l, H, D), g, 1.0, "bf16").pin_memory() for _ in range(3)]
+            for _ in range(steps)]
+    outs = [(torch.empty((P, S_l, H, D), dtype=torch.bfloat16).pin_memory(),
+             torch.empty((P, H // P, P * S_l)).pin_memory()) for _ in range(steps)]
+    passes = [cp.UlyssesHostPass(P, S_l, H, D, device=DEV) for _ in range(2)]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    for i in range(steps):
+        passes[i % 2].run(*host[i], *outs[i], stream=streams[i % 2])
+    torch.cuda.synchronize()
+    for i in range(steps):
+        o_d, l_d = cp.ulysses_fwd(*(t.to(DEV) for t in host[i]), P)
+        torch.cuda.synchronize()
+        assert torch.equal(outs[i][0], o_d.cpu()) and torch.equal(outs[i][1], l_d.cpu()), i
+
+
 def test_ulysses_host_pass_full_size():
     w = W.WORKLOADS[4]
     x = W.make_inputs(w)
