@@ -50,6 +50,10 @@ ATTN_TRAFFIC = {
         "sources_sha256": "cc22e897df40d9a9c09c6b9ba50ff18a9d41e189c17771a08374b346356edc3d",
         "bytes": 594_595_584 + 169_908_224,
     },
+    "attn_fwd_sm100_kernel<128,0,0>": {  # the plain form, in the 5-launch step
+        "sources_sha256": "cc22e897df40d9a9c09c6b9ba50ff18a9d41e189c17771a08374b346356edc3d",
+        "bytes": 571_694_592 + 168_004_608,
+    },
 }
 AUX_REPS = 15  # bursts per auxiliary measurement (median reported, with the range)
 AUX_IDLE_S = 1.0  # idle between the timed steps and the auxiliary measurements
