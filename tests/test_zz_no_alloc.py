@@ -56,6 +56,9 @@ CASES = [
     # 8 ranges over 256 keys would need 65 MiB of partials; the call lowers the split to
     # the two 128-key blocks there are, and two ranges fit in the scratch
     (1, 8, 4096, 256, 128, 8, 2),
+    # n_split = 0: only the items of the last, partial wave of CTAs are split (352 items on
+    # 148 SMs leave 56, each computed as two key ranges)
+    (1, 16, 5520, 2000, 128, 0, 0),
 ]
 
 
