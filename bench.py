@@ -21,6 +21,7 @@ import argparse
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -40,18 +41,19 @@ UNIT = "TFLOP/s"
 WORKLOAD = W.WORKLOADS[4]
 # DRAM bytes (read + write) per launch of each attention kernel on this workload, from one
 # ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the kernel and by the
-# SHA-256 of the kernel sources the capture was taken with.  When the sources hash to
-# something else the figure no longer describes the kernel that runs, and the line reports
-# traffic null until a new capture is recorded here.
+# SHA-256 of the kernel sources the capture was taken with, comments and whitespace removed
+# (an edit to either leaves the kernel as it was).  When the code hashes to something else
+# the figure no longer describes the kernel that runs, and the line reports traffic null
+# until a new capture is recorded here.
 ATTN_SOURCES = ("context_long_sequence_non_b200/csrc/attn_sm100.cu",
                 "context_long_sequence_non_b200/csrc/sm100_ptx.cuh")
 ATTN_TRAFFIC = {
     "attn_fwd_sm100_kernel<128,0,2>": {  # the fused Ulysses kernel, one launch per step
-        "sources_sha256": "cc22e897df40d9a9c09c6b9ba50ff18a9d41e189c17771a08374b346356edc3d",
+        "sources_sha256": "ea5b7c0fb489155c8ff3494afb99ffc8aca83f3006d1b33331772d07d17431f0",
         "bytes": 594_595_584 + 169_908_224,
     },
     "attn_fwd_sm100_kernel<128,0,0>": {  # the plain form, in the 5-launch step
-        "sources_sha256": "cc22e897df40d9a9c09c6b9ba50ff18a9d41e189c17771a08374b346356edc3d",
+        "sources_sha256": "ea5b7c0fb489155c8ff3494afb99ffc8aca83f3006d1b33331772d07d17431f0",
         "bytes": 571_694_592 + 168_004_608,
     },
 }
@@ -61,13 +63,20 @@ L2_NOTE = ("inputs larger than L2: each step streams 543 MB of Q/K/V shards plus
            "permute traffic through the 126 MB L2")
 
 
+def code_only(text):
+    """C/C++/CUDA source with its comments and all whitespace removed."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return re.sub(r"\s+", "", text)
+
+
 def attn_sources_sha256():
     import hashlib
 
     h = hashlib.sha256()
     for rel in ATTN_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            h.update(code_only(f.read()).encode())
     return h.hexdigest()
 
 

@@ -52,7 +52,9 @@ constexpr int kWarpProducer = 8;
 constexpr int kWarpMma = 9;
 // Register split (setmaxnreg): the CTA launches with 168 x 384 = 64512 registers; the two
 // softmax warpgroups take 216 each per thread and the producer/MMA warpgroup 72:
-// 2 x 128 x 216 + 128 x 72 = 64512 (no spills at this split; 56 spills in the issuer).
+// 2 x 128 x 216 + 128 x 72 = 64512.  ptxas reports no spills for D = 64 and an 8-byte
+// stack slot for D = 128 (8 B stored, 24 B loaded, in the producer/issuer warps' code,
+// outside the per-key-block loop of the softmax warps).
 constexpr uint32_t kRegsLaunch = 168, kRegsSoftmax = 216, kRegsOther = 72;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kRegsLaunch * kThreads,
               "register split exceeds the launch allocation");
@@ -401,80 +403,80 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (in_range) ws_lse[wrow] = lse_out;
       } else {
-      if constexpr (kAcc) {
-        // Ring Attention step fused into the epilogue: merge (O_c, LSE_c) into the running
-        // (O_acc, LSE_acc) in place; an empty accumulator (LSE_acc = -inf) takes O_c
-        if (in_range) {
-          const float la2 = (kPreload ? la_pre : lse[lse_idx]) * kLog2e;
-          const float mx = fmaxf(la2, lc2);
-          const float wa = exp2f(la2 - mx), wc = exp2f(lc2 - mx);
-          const float tot = wa + wc;
-          fa = wa / tot;
-          fc = wc / (tot * l);
-          lse_out = (mx + log2f(tot)) * kLn2;
+        if constexpr (kAcc) {
+          // Ring Attention step fused into the epilogue: merge (O_c, LSE_c) into the running
+          // (O_acc, LSE_acc) in place; an empty accumulator (LSE_acc = -inf) takes O_c
+          if (in_range) {
+            const float la2 = (kPreload ? la_pre : lse[lse_idx]) * kLog2e;
+            const float mx = fmaxf(la2, lc2);
+            const float wa = exp2f(la2 - mx), wc = exp2f(lc2 - mx);
+            const float tot = wa + wc;
+            fa = wa / tot;
+            fc = wc / (tot * l);
+            lse_out = (mx + log2f(tot)) * kLn2;
+          }
         }
-      }
-      // one 32-column chunk of the row: scaled (and merged into the accumulator) and stored
-      auto store_chunk = [&](int c, const uint32_t (&r)[32]) {
-        if (!in_range) return;
-        if constexpr (kOutF32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + row_off + c * 32);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            float4 v = make_float4(__uint_as_float(r[4 * e]) * fc, __uint_as_float(r[4 * e + 1]) * fc,
-                                   __uint_as_float(r[4 * e + 2]) * fc, __uint_as_float(r[4 * e + 3]) * fc);
-            if (kAcc && fa != 0.f) {  // an empty accumulator row is never read
-              const float4 a = dst[e];
-              v.x = fmaf(fa, a.x, v.x);
-              v.y = fmaf(fa, a.y, v.y);
-              v.z = fmaf(fa, a.z, v.z);
-              v.w = fmaf(fa, a.w, v.w);
+        // one 32-column chunk of the row: scaled (and merged into the accumulator) and stored
+        auto store_chunk = [&](int c, const uint32_t (&r)[32]) {
+          if (!in_range) return;
+          if constexpr (kOutF32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + row_off + c * 32);
+  #pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              float4 v = make_float4(__uint_as_float(r[4 * e]) * fc, __uint_as_float(r[4 * e + 1]) * fc,
+                                     __uint_as_float(r[4 * e + 2]) * fc, __uint_as_float(r[4 * e + 3]) * fc);
+              if (kAcc && fa != 0.f) {  // an empty accumulator row is never read
+                const float4 a = dst[e];
+                v.x = fmaf(fa, a.x, v.x);
+                v.y = fmaf(fa, a.y, v.y);
+                v.z = fmaf(fa, a.z, v.z);
+                v.w = fmaf(fa, a.w, v.w);
+              }
+              dst[e] = v;
             }
-            dst[e] = v;
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + row_off + c * 32);
+  #pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float o[8];
+  #pragma unroll
+              for (int t = 0; t < 8; ++t) o[t] = __uint_as_float(r[8 * e + t]) * fc;
+              if (kAcc && fa != 0.f) {  // an empty accumulator's row is not used
+                uint4 a;
+                if constexpr (kPreload) a = acc_row[c * 4 + e];
+                else a = dst[e];
+                const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+  #pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                  o[2 * t] = fmaf(fa, __uint_as_float(aw[t] << 16), o[2 * t]);
+                  o[2 * t + 1] = fmaf(fa, __uint_as_float(aw[t] & 0xFFFF0000u), o[2 * t + 1]);
+                }
+              }
+              uint4 v;
+              v.x = pack_bf16x2(o[0], o[1]);
+              v.y = pack_bf16x2(o[2], o[3]);
+              v.z = pack_bf16x2(o[4], o[5]);
+              v.w = pack_bf16x2(o[6], o[7]);
+              dst[e] = v;
+            }
+          }
+        };
+        if constexpr (kPreload) {
+  #pragma unroll
+          for (int c = 0; c < D / 32; ++c) {  // unrolled: acc_row is indexed statically
+            uint32_t r[32];
+            tmem_ld32(t_o + c * 32, r);
+            store_chunk(c, r);
           }
         } else {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + row_off + c * 32);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float o[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t) o[t] = __uint_as_float(r[8 * e + t]) * fc;
-            if (kAcc && fa != 0.f) {  // an empty accumulator's row is not used
-              uint4 a;
-              if constexpr (kPreload) a = acc_row[c * 4 + e];
-              else a = dst[e];
-              const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-              for (int t = 0; t < 4; ++t) {
-                o[2 * t] = fmaf(fa, __uint_as_float(aw[t] << 16), o[2 * t]);
-                o[2 * t + 1] = fmaf(fa, __uint_as_float(aw[t] & 0xFFFF0000u), o[2 * t + 1]);
-              }
-            }
-            uint4 v;
-            v.x = pack_bf16x2(o[0], o[1]);
-            v.y = pack_bf16x2(o[2], o[3]);
-            v.z = pack_bf16x2(o[4], o[5]);
-            v.w = pack_bf16x2(o[6], o[7]);
-            dst[e] = v;
+  #pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(t_o + c * 32, r);
+            store_chunk(c, r);
           }
         }
-      };
-      if constexpr (kPreload) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {  // unrolled: acc_row is indexed statically
-          uint32_t r[32];
-          tmem_ld32(t_o + c * 32, r);
-          store_chunk(c, r);
-        }
-      } else {
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(t_o + c * 32, r);
-          store_chunk(c, r);
-        }
-      }
-      if (in_range && lse != nullptr) lse[lse_idx] = lse_out;
+        if (in_range && lse != nullptr) lse[lse_idx] = lse_out;
       }
     }
   } else {

@@ -29,3 +29,25 @@ def test_reference_arm_json_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["e2e"]["value"] == d["value"] and d["e2e"]["unit"] == d["unit"]
+
+
+def _bench_module():
+    import importlib.util
+
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_traffic_hash_ignores_comments_and_whitespace_only():
+    bench = _bench_module()
+    src = "int f(int a) {  // add one\n  return a + 1; /* done\n  here */\n}\n"
+    same = "int f(int a)\n{\n\treturn a+1;  // different words\n}"
+    other = "int f(int a) { return a + 2; }"
+    assert bench.code_only(src) == bench.code_only(same) == "intf(inta){returna+1;}"
+    assert bench.code_only(other) != bench.code_only(src)
+    # every recorded capture names a kernel that bench.py times and a full SHA-256
+    for kernel, rec in bench.ATTN_TRAFFIC.items():
+        assert kernel.startswith("attn_fwd_sm100_kernel<")
+        assert len(rec["sources_sha256"]) == 64 and rec["bytes"] > 0
