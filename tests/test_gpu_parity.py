@@ -187,17 +187,17 @@ def test_bf16_shapes_match_oracle(shape):
     assert rel_l2(o32, o_ref) < 1e-2
 
 
-# The attention kernel is persistent: at most one CTA per SM (148 on B200) loops over work
-# items of (256-row query tile pair, head, batch).  These shapes give CTAs several items
-# each, with ragged query and key tails, single-block items and both head widths, so that
-# the pipeline's hand-over from one item to the next (Q reload, O read-out while the next
-# item's S is computed) is checked element by element.
+# The attention kernel runs one CTA per work item of (256-row query tile pair, head, batch),
+# one CTA per SM at a time (148 on B200).  These shapes give grids of more items than SMs
+# (several waves, a partial last wave), with ragged query and key tails, single-block items
+# and both head widths, so that every item's addressing -- and the SM's hand-over from one
+# CTA to the next -- is checked element by element.
 MULTI_ITEM_SHAPES = [(2, 40, 300, 257, 128), (1, 96, 600, 130, 64), (1, 150, 256, 100, 128),
                      (3, 70, 513, 384, 128)]
 
 
 @pytest.mark.parametrize("shape", MULTI_ITEM_SHAPES)
-def test_persistent_items_match_oracle(shape):
+def test_multi_wave_items_match_oracle(shape):
     Bn, H, Sq, Skv, D = shape
     q, k, v = W.random_case(7 * Sq + H, Bn, H, Sq, Skv, D)
     scale = 1.0 / math.sqrt(D)
@@ -226,7 +226,7 @@ def test_persistent_items_match_oracle(shape):
     check_lse(l_s, l_ref, f"{shape} split 3")
 
 
-def test_persistent_fused_ulysses_many_items():
+def test_fused_ulysses_many_items():
     # 4 ranks x 400 tokens, 64 heads: 7 tile pairs x 16 heads x 4 groups = 448 items
     P, S_l, H, D = 4, 400, 64, 128
     g = torch.Generator().manual_seed(404)
