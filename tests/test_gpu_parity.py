@@ -40,9 +40,14 @@ def bits(t):
 # ----------------------------------------------------------------------------- permutes
 
 
+# A row (Hp * D * element bytes) moves as 32-vector chunks of 16 bytes: (2, 9, 32, 128) and
+# (1, 5, 4, 256, f32) have 4 KB rows of 8 chunks each, the others one chunk, whole or
+# partial; S_l = 33 and 300 are not multiples of the warps' row steps.
 @pytest.mark.parametrize("P,S_l,H,D,dt", [(2, 3, 4, 8, torch.bfloat16), (4, 5, 8, 16, torch.float32),
                                           (1, 7, 2, 64, torch.bfloat16), (8, 33, 16, 128, torch.bfloat16),
-                                          (3, 10, 6, 8, torch.bfloat16), (2, 1, 2, 8, torch.float32)])
+                                          (3, 10, 6, 8, torch.bfloat16), (2, 1, 2, 8, torch.float32),
+                                          (3, 300, 6, 64, torch.float32), (2, 9, 32, 128, torch.bfloat16),
+                                          (1, 5, 4, 256, torch.float32)])
 def test_permutes_bit_exact(P, S_l, H, D, dt):
     g = torch.Generator().manual_seed(P * 1000 + S_l)
     ib = torch.int16 if dt == torch.bfloat16 else torch.int32
@@ -69,7 +74,7 @@ def test_permutes_ulysses_full_size_bit_exact():
     assert torch.equal(bits(back).cpu(), src_bits)
 
 
-@pytest.mark.parametrize("P,S_l,H,D", [(2, 3, 4, 8), (8, 5520, 16, 128), (3, 7, 6, 16)])
+@pytest.mark.parametrize("P,S_l,H,D", [(2, 3, 4, 8), (8, 5520, 16, 128), (3, 7, 6, 16), (2, 9, 32, 128)])
 def test_seq2head_qkv_batched_bit_exact(P, S_l, H, D):
     g = torch.Generator().manual_seed(P + S_l)
     srcs = [torch.randint(-32768, 32768, (P, S_l, H, D), generator=g, dtype=torch.int32).to(torch.int16)

@@ -91,8 +91,10 @@ def test_rmsnorm_zero_rows_and_zero_input():
     assert torch.equal(bits(y), bits(z))
 
 
+# (1, 9, 4, 256) has 2 KB rows (4 chunks of 32 vectors) and (2, 11, 24, 128) 3 KB rows
+# (6 chunks): head rows in every chunk position.
 @pytest.mark.parametrize("P,S_l,H,D", [(2, 3, 4, 8), (4, 33, 8, 128), (8, 17, 16, 128),
-                                       (2, 5, 2, 64), (1, 9, 4, 256), (3, 7, 6, 32)])
+                                       (2, 5, 2, 64), (1, 9, 4, 256), (3, 7, 6, 32), (2, 11, 24, 128)])
 def test_seq2head_qkv_norm_matches_oracle(P, S_l, H, D):
     g = torch.Generator().manual_seed(P * 31 + S_l)
     q, k, v = (W.randn((P, S_l, H, D), g, 3.0, "bf16") for _ in range(3))
