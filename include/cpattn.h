@@ -25,6 +25,13 @@
  *     pointers 4-byte aligned (CPATTN_ERR_ALIGN otherwise).
  *   - Every argument is checked before the first CUDA call, so argument errors are
  *     reported the same way with or without a GPU.
+ *   - Stream capture: a call that takes a stream only launches kernels on it (kernels
+ *     launched as programmatic dependents of the previous one), so it can be recorded
+ *     into a CUDA graph and replayed; the graph keeps the pointers and sizes of the
+ *     recorded call.  Make one ordinary call first: the first call on a device loads the
+ *     module and looks up the device error word.  Not capturable: cpattn_ulysses_host
+ *     (its own streams and events), cpattn_device_error (synchronises the device), and
+ *     the first cpattn_fwd_split_noalloc call on a device (see there).
  */
 #ifndef CPATTN_H
 #define CPATTN_H
