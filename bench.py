@@ -584,6 +584,20 @@ def next_paths(cp, w, q, k, v, plan, dev, stream):
                                            n_split=n_split))
     ms_t = timed(lambda: cp.ring_attention(q3, kc, vc, scale=w3.softmax_scale, fused=True,
                                            n_split=0))
+    # the same tail-split step recorded once into a CUDA graph and replayed, as a serving
+    # loop runs it (no host work between its launches)
+    ring_t = lambda: cp.ring_attention(q3, kc, vc, scale=w3.softmax_scale, fused=True, n_split=0)
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        ring_t()
+    stream.wait_stream(side)
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        ring_t()
+    ms_g = timed(graph.replay)
+    del graph
     # AllGather-KV-like: a short query slice (512 tokens, 16 heads) against all 44160 keys --
     # 32 CTAs for 148 SMs, the case split-KV is for
     g = torch.Generator(device="cpu").manual_seed(41)
@@ -610,6 +624,9 @@ def next_paths(cp, w, q, k, v, plan, dev, stream):
         "tail_split_frac_of_burst": round(w3.attn_flops / ms_t / 1e9 / peaks["bf16_tflops"], 4),
         "tail_split": ("352 items on 148 SMs: 296 whole, the 56 of the last wave as 2 key "
                        "ranges each, folded into the accumulator by a combine kernel"),
+        "tail_split_graph_ms": round(ms_g, 4),
+        "tail_split_graph_TFLOP/s": round(w3.attn_flops / ms_g / 1e9, 2),
+        "tail_split_graph_frac_of_burst": round(w3.attn_flops / ms_g / 1e9 / peaks["bf16_tflops"], 4),
         "launches_fused": 8, "launches_unfused": 15, "launches_split": 16,
         "launches_tail_split": 16}
     return res
