@@ -376,7 +376,7 @@ def run_ours(args, world, rank, local):
         aux["clocks"] = aux_clocks.stop(wall_a0, time.time())
         aux["idle_before_s"] = AUX_IDLE_S
         # ---- end to end through the public API with host buffers
-        e2e = e2e_run(cp, UlyssesPlan, w, x, dev, stream, args)
+        e2e = e2e_run(cp, UlyssesPlan, w, x, dev, stream, args, dist=dist, world=world)
 
     hr = results[head]
     max_ms, total_flops, attn_ms = hr.pop("_raw")
@@ -632,7 +632,7 @@ def next_paths(cp, w, q, k, v, plan, dev, stream):
     return res
 
 
-def e2e_run(cp, UlyssesPlan, w, x, dev, stream, args):
+def e2e_run(cp, UlyssesPlan, w, x, dev, stream, args, dist=None, world=1):
     """Same metric end to end with pinned host buffers: every step copies its Q/K/V shards
     host -> device and its O and LSE device -> host inside the timed region.
 
@@ -691,6 +691,9 @@ def e2e_run(cp, UlyssesPlan, w, x, dev, stream, args):
             host_step()
         torch.cuda.synchronize(dev)
         kk[0] = 0
+        if dist is not None:  # every rank's timed region starts together
+            dist.barrier()
+            torch.cuda.synchronize(dev)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(n):
@@ -703,6 +706,10 @@ def e2e_run(cp, UlyssesPlan, w, x, dev, stream, args):
 
     ms_host = host_timed()
     del hps
+    # the whole job: the max of the ranks' timed regions, the work and copies of all ranks
+    ms_all, flops_all = aggregate(dist, ms_host * n, w.attn_flops * n,
+                                  device=dev if dist is not None else None)
+    ms_job = ms_all / n
 
     dq, dk, dv = (torch.empty_like(hq, device=dev) for _ in range(3))
 
@@ -727,12 +734,14 @@ def e2e_run(cp, UlyssesPlan, w, x, dev, stream, args):
         k[0] += 1
 
     ms_streamer = timed(stream_step, streamer.upload, streamer.download)
-    return {"value": tf(ms_host), "unit": UNIT, "ms_per_step": round(ms_host, 4),
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
+    return {"value": round(flops_all / n / (ms_job * 1e-3) / 1e12, 2), "unit": UNIT,
+            "ms_per_step": round(ms_job, 4), "n_gpus": world,
+            "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": d2h * world, "steps": n,
             "mode": ("C ABI cpattn_ulysses_host (UlyssesHostPass): pinned host Q/K/V shards in, "
                      "host O + LSE out; one chunk per head group (8), uploads and downloads "
                      "overlapping the attention inside each call; two passes alternating on "
                      "two streams (double-buffered serving loop)"),
+            "per_rank": "single_stream, streamer and serial are this rank's own (rank 0)",
             "single_stream": {"value": tf(ms_single), "ms_per_step": round(ms_single, 4),
                               "mode": "the same call back to back on one stream"},
             "streamer": {"value": tf(ms_streamer), "ms_per_step": round(ms_streamer, 4),
