@@ -401,7 +401,8 @@ def run_ours(args, world, rank, local):
             "peak_kind": (f"{peaks['source']} cuBLAS bf16 "
                           f"{'sustained' if long_run else 'burst'}"),
             "algorithmic_flops_per_launch": flops,
-            "avg_launch_ms": round(attn_ms, 4), "traffic": attn_traffic(kernel),
+            "avg_launch_ms": round(attn_ms, 4),
+            "traffic": attn_traffic(kernel),
             "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
             "traffic_source": ("ncu capture of this kernel, recorded with the SHA-256 of its "
                                "sources; null when the sources have changed since"),
@@ -548,7 +549,15 @@ def next_paths(cp, w, q, k, v, plan, dev, stream):
     del q5, k5, v5, x5
     ms = timed(lambda: cp.ulysses_fwd(q, k, v, w.P, out=plan.out, lse=plan.lse))
     res["ulysses_fused"] = {"ms": round(ms, 4), "TFLOP/s": round(w.attn_flops / ms / 1e9, 2),
-                            "what": "seq2head x3 + attention + head2seq as one kernel"}
+                            "what": ("seq2head x3 + attention + head2seq as one kernel "
+                                     "(cpattn_ulysses_fwd, no tail split)")}
+    ws_u = torch.empty(max(cp.ulysses_workspace_bytes(w.P, w.Sq // w.P, w.H * w.P, w.D), 256),
+                       dtype=torch.uint8, device=dev)
+    ms = timed(lambda: cp.ulysses_fwd_split(q, k, v, w.P, out=plan.out, lse=plan.lse,
+                                            workspace=ws_u))
+    res["ulysses_fused_split"] = {"ms": round(ms, 4), "TFLOP/s": round(w.attn_flops / ms / 1e9, 2),
+                                  "what": "the same with the tail split (cpattn_ulysses_fwd_split)"}
+    del ws_u
     ms = timed(lambda: cp.seq2head_qkv(q, k, v, w.P, out=(plan.qh, plan.kh, plan.vh)))
     nbytes = 3 * 2 * q.numel() * q.element_size()
     res["seq2head_qkv"] = {"ms": round(ms, 4), "bytes": nbytes,

@@ -23,6 +23,8 @@ from ._binding import (  # noqa: F401
     split_suggest,
     split_workspace_bytes,
     ulysses_fwd,
+    ulysses_fwd_split,
+    ulysses_workspace_bytes,
     ulysses_host,
     head2seq,
     lib,

@@ -49,6 +49,10 @@ def lib() -> ctypes.CDLL:
             L.cpattn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
             L.cpattn_fwd_accumulate.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
             L.cpattn_ulysses_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+            L.cpattn_ulysses_fwd_split.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp,
+                                                   ctypes.c_size_t, vp]
+            L.cpattn_ulysses_fwd_workspace.argtypes = [i, i, i, i, i]
+            L.cpattn_ulysses_fwd_workspace.restype = ctypes.c_size_t
             L.cpattn_ulysses_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i,
                                               f, i, i, vp]
             L.cpattn_fwd_split.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp,
@@ -70,7 +74,7 @@ def lib() -> ctypes.CDLL:
             L.cpattn_version.argtypes = []
             L.cpattn_selftest_exp2.argtypes = [vp, vp, i, vp]
             for name in ("cpattn_fwd", "cpattn_fwd_accumulate", "cpattn_ulysses_fwd",
-                         "cpattn_ulysses_host",
+                         "cpattn_ulysses_fwd_split", "cpattn_ulysses_host",
                          "cpattn_fwd_split", "cpattn_split_suggest", "cpattn_merge", "cpattn_seq2head_qkv", "cpattn_seq2head", "cpattn_head2seq",
                          "cpattn_device_error", "cpattn_selftest_wait_timeout", "cpattn_version",
                          "cpattn_selftest_exp2"):
@@ -158,6 +162,38 @@ def ulysses_fwd(q, k, v, P, out=None, lse=None, scale=None, out_dtype=None, want
     st = lib().cpattn_ulysses_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), P, S_l, H, D,
                                   float(scale), _dtype_code(out.dtype), _stream(stream))
     _check(st, "cpattn_ulysses_fwd")
+    return out, lse
+
+
+def ulysses_workspace_bytes(P, S_l, H, D, out_dtype=torch.bfloat16) -> int:
+    """Workspace bytes of ulysses_fwd_split for these shards (0: nothing to split)."""
+    return int(lib().cpattn_ulysses_fwd_workspace(P, S_l, H, D, _dtype_code(out_dtype)))
+
+
+def ulysses_fwd_split(q, k, v, P, out=None, lse=None, scale=None, out_dtype=None,
+                      want_lse=True, workspace=None, stream=None):
+    """ulysses_fwd with the tail split (the items of the GPU's last wave or two computed
+    as key ranges and folded exactly).  ``workspace``: a uint8 CUDA tensor of at least
+    ``ulysses_workspace_bytes(...)`` bytes, allocated here (by PyTorch) when omitted."""
+    P_, S_l, H, D = q.shape
+    if P_ != P or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must be same-shaped [P][S_l][H][D] shards")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty((P, S_l, H, D), dtype=out_dtype or q.dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((P, H // P, P * S_l), dtype=torch.float32, device=q.device)
+    need = ulysses_workspace_bytes(P, S_l, H, D, out.dtype)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _need_cuda(q, k, v, out, lse, workspace)
+    st = lib().cpattn_ulysses_fwd_split(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), P, S_l,
+                                        H, D, float(scale), _dtype_code(out.dtype),
+                                        _ptr(workspace),
+                                        workspace.numel() if workspace is not None else 0,
+                                        _stream(stream))
+    _check(st, "cpattn_ulysses_fwd_split")
     return out, lse
 
 

@@ -182,10 +182,10 @@ size_t cpattn_fwd_split_workspace(int B, int H, int Sq, int D, int n_split, int 
   if (B < 1 || H < 1 || Sq < 1 || D < 1 || n_split < 0 || n_split > kMaxSplit || es == 0)
     return 0;
   if (n_split == 0) {
-    // tail split: the plan depends on the key count only through "at least 2 blocks per
-    // range"; size the workspace for the most parts any key count can give
+    // tail split: the plan depends on the key count, which this query does not take; size
+    // the workspace for the largest plan any key count can give
     if (D != 64 && D != 128) return 0;
-    return cpattn::tail_split_workspace(cpattn::tail_split_plan(B, H, Sq, 1 << 30), D);
+    return cpattn::tail_split_workspace_bound(B, H, Sq, D);
   }
   return n_split == 1 ? 0 : split_ws_bytes(B, H, Sq, D, n_split, es);
 }
@@ -220,7 +220,7 @@ int cpattn_fwd_split(const void* q, const void* k, const void* v, void* out, flo
   if (n_split < 0 || n_split > kMaxSplit) return CPATTN_ERR_SHAPE;
   const int n_kv = Skv > 0 ? (Skv + 127) / 128 : 0;
   cpattn::TailSplit tail{};
-  if (n_split == 0) {  // tail split: only the items of the last, partial wave are split
+  if (n_split == 0) {  // tail split: only the items of the last wave or two are split
     if (B >= 1 && H >= 1 && Sq >= 1 && Skv >= 1) tail = cpattn::tail_split_plan(B, H, Sq, Skv);
     if (tail.parts < 2) n_split = 1;
   } else if (n_split > n_kv) {
@@ -361,6 +361,48 @@ int cpattn_ulysses_fwd(const void* q, const void* k, const void* v, void* out, f
       m.q, m.k, m.v, m.q16, m.k16, m.v16, out, lse, P, S_local, H, D, scale_log2,
       cpattn::kRescaleLog2, out_dtype == CPATTN_F32, 0, P, err, cpattn::kDefaultWaitLimit,
       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t cpattn_ulysses_fwd_workspace(int P, int S_local, int H, int D, int out_dtype) {
+  if (P < 1 || S_local < 1 || H < 1 || H % P != 0 || elem_size(out_dtype) == 0) return 0;
+  if ((D != 64 && D != 128) || (long long)P * S_local > 0x7fffffffLL) return 0;
+  const int S = P * S_local;
+  return cpattn::tail_split_workspace(cpattn::tail_split_plan(P, H / P, S, S), D);
+}
+
+int cpattn_ulysses_fwd_split(const void* q, const void* k, const void* v, void* out, float* lse,
+                             int P, int S_local, int H, int D, float scale, int out_dtype,
+                             void* workspace, size_t workspace_bytes, cpattn_stream_t stream) {
+  const int st = ulysses_args(q, k, v, out, lse, P, S_local, H, D, scale, out_dtype);
+  if (st != CPATTN_OK) return st;
+  const int S = P * S_local;
+  const cpattn::TailSplit tail = cpattn::tail_split_plan(P, H / P, S, S);
+  const size_t need = cpattn::tail_split_workspace(tail, D);
+  if (need > 0) {
+    if (workspace == nullptr) return CPATTN_ERR_NULL;
+    if (!aligned(workspace, 256)) return CPATTN_ERR_ALIGN;
+    if (workspace_bytes < need) return CPATTN_ERR_SHAPE;
+    const size_t io = size_t(S) * H * D;
+    const int es = elem_size(out_dtype);
+    if (overlap(workspace, need, q, io * 2) || overlap(workspace, need, k, io * 2) ||
+        overlap(workspace, need, v, io * 2) || overlap(workspace, need, out, io * es) ||
+        (lse != nullptr && overlap(workspace, need, lse, size_t(H) * S * 4)))
+      return CPATTN_ERR_SHAPE;
+  }
+  int* err = device_error_word();
+  if (err == nullptr) return CPATTN_ERR_CUDA;
+  UlyssesMaps m;
+  if (!encode_ulysses(&m, q, k, v, P, S_local, H, D)) return CPATTN_ERR_CUDA;
+  const float scale_log2 = float(double(scale) * 1.4426950408889634074);
+  const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (need == 0)
+    return cuda_status(cpattn::launch_ulysses_fwd_sm100(
+        m.q, m.k, m.v, m.q16, m.k16, m.v16, out, lse, P, S_local, H, D, scale_log2,
+        cpattn::kRescaleLog2, out_dtype == CPATTN_F32, 0, P, err, cpattn::kDefaultWaitLimit, cs));
+  return cuda_status(cpattn::launch_ulysses_fwd_sm100_tail(
+      m.q, m.k, m.v, m.q16, m.k16, m.v16, out, lse, P, S_local, H, D, scale_log2,
+      cpattn::kRescaleLog2, out_dtype == CPATTN_F32, tail, workspace, err,
+      cpattn::kDefaultWaitLimit, cs));
 }
 
 int cpattn_ulysses_host(const void* h_q, const void* h_k, const void* h_v, void* h_out,

@@ -703,25 +703,61 @@ cudaError_t launch_any(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
 
 }  // namespace
 
+// Candidate tail splits: the last rem + k * sms work items (k = 0: the partial last wave
+// alone; k = 1: that wave and the whole wave before it) as p key ranges each, the rest
+// whole.  p <= 8 for k = 0 and p <= 4 for k = 1, which bounds the workspace.
+constexpr int kTailMaxParts[2] = {8, 4};
+
 TailSplit tail_split_plan(int B, int H, int Sq, int Skv) {
   TailSplit t{};
   const long long pairs = (Sq + 2 * kBlockM - 1) / (2 * kBlockM);
   const long long items = pairs * H * B;
   const int sms = sm_count();
   const int n_kv = (Skv + kBlockN - 1) / kBlockN;
-  if (items < 1 || items > 0x7fffffffLL || n_kv < 2) return t;
+  if (items < 1 || items > 0x7fffffffLL || n_kv < 4) return t;
   const long long rem = items % sms;  // items of the last, partial wave
   if (rem == 0) return t;
-  // split each of them into as many key ranges as still fit in one wave (at most 8, and
-  // at least 2 key blocks per range)
-  long long parts = sms / rem;
-  if (parts > 8) parts = 8;
-  if (parts > n_kv / 2) parts = n_kv / 2;
-  if (parts < 2) return t;
-  t.n_full = int(items - rem);
-  t.n_tail = int(rem);
-  t.parts = int(parts);
+  // Makespan in units of one whole item's time, each CTA paying a fixed start-up and
+  // epilogue of about two key blocks (c): whole waves cost 1 + c, and the split items'
+  // ranges run in ceil(tail * p / sms) short waves of 1/p + c.  Split only when that saves
+  // at least 0.5 %.
+  const double c = 2.0 / n_kv;
+  const double whole = double((items + sms - 1) / sms) * (1.0 + c);
+  double best = whole * 0.995;
+  for (int k = 0; k < 2; ++k) {
+    const long long tail = rem + (long long)k * sms;
+    if (tail > items) break;
+    const double before = double((items - tail) / sms) * (1.0 + c);
+    for (int p = 2; p <= kTailMaxParts[k] && p <= n_kv / 2; ++p) {
+      const long long short_waves = (tail * p + sms - 1) / sms;
+      const double span = before + double(short_waves) * (1.0 / p + c);
+      if (span < best) {
+        best = span;
+        t.n_full = int(items - tail);
+        t.n_tail = int(tail);
+        t.parts = p;
+      }
+    }
+  }
   return t;
+}
+
+size_t tail_split_workspace_bound(int B, int H, int Sq, int D) {
+  const long long pairs = (Sq + 2 * kBlockM - 1) / (2 * kBlockM);
+  const long long items = pairs * H * B;
+  const int sms = sm_count();
+  if (items < 1 || items > 0x7fffffffLL || items % sms == 0) return 0;
+  TailSplit t{};
+  long long worst = 0;
+  for (int k = 0; k < 2; ++k) {
+    const long long tail = items % sms + (long long)k * sms;
+    if (tail <= items && tail * kTailMaxParts[k] > worst) {
+      worst = tail * kTailMaxParts[k];
+      t.n_tail = int(tail);
+      t.parts = kTailMaxParts[k];
+    }
+  }
+  return tail_split_workspace(t, D);
 }
 
 size_t tail_split_workspace(const TailSplit& t, int D) {
@@ -763,7 +799,34 @@ cudaError_t launch_attn_fwd_sm100_tail(const CUtensorMap& tq, const CUtensorMap&
                              accumulate ? kAccum : kPlain, stream);
   if (e != cudaSuccess) return e;
   return launch_combine_tail(a.ws_o, a.ws_lse, t.n_full, t.n_tail, t.parts, out, lse, B, H, Sq,
-                             D, out_f32 ? 4 : 2, accumulate, stream);
+                             D, out_f32 ? 4 : 2, accumulate, /*batch_stride=*/Sq * H,
+                             /*token_stride=*/H, stream);
+}
+
+cudaError_t launch_ulysses_fwd_sm100_tail(const CUtensorMap& tq, const CUtensorMap& tk,
+                                          const CUtensorMap& tv, const CUtensorMap& tq16,
+                                          const CUtensorMap& tk16, const CUtensorMap& tv16,
+                                          void* out, float* lse, int P, int S_local, int H, int D,
+                                          float scale_log2, float rescale_log2, bool out_f32,
+                                          const TailSplit& t, void* workspace, int* err,
+                                          long long wait_limit, cudaStream_t stream) {
+  const int S = P * S_local, Hp = H / P;
+  const size_t rows = size_t(t.parts) * t.n_tail * (2 * kBlockM);
+  Launch a{};
+  a.grid = dim3(unsigned(t.n_full + t.n_tail * t.parts), 1, 1);
+  a.H = Hp, a.Sq = S, a.Skv = S, a.s_local = S_local, a.n_split = 1, a.b_first = 0;
+  a.n_full = t.n_full, a.n_tail = t.n_tail, a.tail_parts = t.parts;
+  a.ws_o = static_cast<float*>(workspace);
+  a.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                      ((rows * D * 4 + 255) & ~size_t(255)));
+  a.scale_log2 = scale_log2, a.rescale_log2 = rescale_log2, a.err = err, a.wait_limit = wait_limit;
+  cudaError_t e = launch_any(tq, tk, tv, tq16, tk16, tv16, out, lse, D, a, out_f32, kSharded,
+                             stream);
+  if (e != cudaSuccess) return e;
+  // token q of head group g, head j: row q of the flattened [P][S_local] shards, head g*Hp + j
+  return launch_combine_tail(a.ws_o, a.ws_lse, t.n_full, t.n_tail, t.parts, out, lse, P, Hp, S,
+                             D, out_f32 ? 4 : 2, false, /*batch_stride=*/Hp, /*token_stride=*/H,
+                             stream);
 }
 
 cudaError_t launch_ulysses_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,

@@ -24,13 +24,17 @@ cudaError_t launch_attn_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk,
 
 // Tail split of a single-pass attention launch: the first n_full work items (256-row tile
 // pair x head x batch; whole waves of one CTA per SM) run over all keys, the last n_tail
-// items each as `parts` key ranges whose fp32 partials go to a workspace and are folded by
-// a combine kernel.  parts < 2: nothing to gain, run the plain launch.
+// items -- the partial last wave, or that wave and the whole one before it -- each as
+// `parts` key ranges whose fp32 partials go to a workspace and are folded by a combine
+// kernel.  The plan minimises the modelled makespan; parts < 2: nothing to gain, run the
+// plain launch.
 struct TailSplit {
   int n_full, n_tail, parts;
 };
 TailSplit tail_split_plan(int B, int H, int Sq, int Skv);
 size_t tail_split_workspace(const TailSplit& t, int D);  // bytes (0 when parts < 2)
+// The largest workspace any key length can make the plan of (B, H, Sq) need.
+size_t tail_split_workspace_bound(int B, int H, int Sq, int D);
 
 // The attention (plain or accumulate) with a tail split, then the combine of the tail
 // items' partials into (out, lse) -- with `accumulate`, merged into the running (out, lse).
@@ -43,9 +47,24 @@ cudaError_t launch_attn_fwd_sm100_tail(const CUtensorMap& tq, const CUtensorMap&
 
 // Fold the tail items' key-range partials (fp32 O rows [parts][n_tail][256][D], LSE
 // [parts][n_tail][256]) -- and with `accumulate` the running (out, lse) -- into out / lse.
+// Row (b, q, h) of out starts at element (b * batch_stride + q * token_stride + h) * D:
+// [B][Sq][H][D] has batch_stride = Sq * H and token_stride = H; the Ulysses shards (b the
+// head group, H its heads) have batch_stride = H and token_stride = H * B.  LSE is
+// [B][H][Sq] either way.
 cudaError_t launch_combine_tail(const float* ws_o, const float* ws_lse, int n_full, int n_tail,
                                 int parts, void* out, float* lse, int B, int H, int Sq, int D,
-                                int out_bytes, bool accumulate, cudaStream_t stream);
+                                int out_bytes, bool accumulate, long long batch_stride,
+                                int token_stride, cudaStream_t stream);
+
+// The fused Ulysses pass over all P head groups with a tail split (work items numbered tile
+// pair fastest, then head, then group), then the combine of the tail items' partials.
+cudaError_t launch_ulysses_fwd_sm100_tail(const CUtensorMap& tq, const CUtensorMap& tk,
+                                          const CUtensorMap& tv, const CUtensorMap& tq16,
+                                          const CUtensorMap& tk16, const CUtensorMap& tv16,
+                                          void* out, float* lse, int P, int S_local, int H, int D,
+                                          float scale_log2, float rescale_log2, bool out_f32,
+                                          const TailSplit& t, void* workspace, int* err,
+                                          long long wait_limit, cudaStream_t stream);
 
 // Ulysses fused: q/k/v/out are [P][S_local][H][D] rank shards, each described by two tensor
 // maps over dims (D, H, S_local, P): a 64 x 1 x 128 x 1 box and a 64 x 1 x 16 x 1 box (for

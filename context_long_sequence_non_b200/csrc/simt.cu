@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(kMergeThreads) combine_kernel(
 template <int VPL, bool kOutBf16, bool kAcc>
 __global__ void __launch_bounds__(256) combine_tail_kernel(
     const float* __restrict__ ws_o, const float* __restrict__ ws_lse, int n_full, int n_tail,
-    int parts, void* out, float* lse, int H, int Sq) {
+    int parts, void* out, float* lse, int H, int Sq, long long batch_stride, int token_stride) {
   dependent_launch_gate();
   constexpr int D = 32 * VPL;
   const int lane = threadIdx.x & 31;
@@ -382,7 +382,8 @@ __global__ void __launch_bounds__(256) combine_tail_kernel(
   const int q = pair * 256 + r;
   if (q >= Sq) return;  // rows past the end of the sequence were never written
   const size_t li = (size_t(b) * H + h) * Sq + q;
-  const size_t orow = ((size_t(b) * Sq + q) * H + h) * D + lane * VPL;
+  const size_t orow =
+      (size_t(b) * batch_stride + size_t(q) * token_stride + h) * D + lane * VPL;
   float lp[8];
   float mx = -INFINITY;
   for (int p = 0; p < parts; ++p) {
@@ -735,7 +736,8 @@ cudaError_t launch_combine(const void* part_o, const float* part_lse, int n, voi
 
 cudaError_t launch_combine_tail(const float* ws_o, const float* ws_lse, int n_full, int n_tail,
                                 int parts, void* out, float* lse, int B, int H, int Sq, int D,
-                                int out_bytes, bool accumulate, cudaStream_t stream) {
+                                int out_bytes, bool accumulate, long long batch_stride,
+                                int token_stride, cudaStream_t stream) {
   (void)B;
   if (parts < 1 || parts > 8 || n_tail < 1 || (D != 64 && D != 128)) return cudaErrorInvalidValue;
   const unsigned blocks = unsigned((n_tail * 256 + 7) / 8);
@@ -746,7 +748,7 @@ cudaError_t launch_combine_tail(const float* ws_o, const float* ws_lse, int n_fu
       : (bf ? (accumulate ? combine_tail_kernel<2, true, true> : combine_tail_kernel<2, true, false>)
             : (accumulate ? combine_tail_kernel<2, false, true> : combine_tail_kernel<2, false, false>));
   return launch_dependent(kernel, dim3(blocks), dim3(256), stream, ws_o, ws_lse, n_full, n_tail,
-                          parts, out, lse, H, Sq);
+                          parts, out, lse, H, Sq, batch_stride, token_stride);
 }
 
 static cudaError_t launch_permute(bool to_head, const void* const* src, void* const* dst,

@@ -104,11 +104,17 @@ CPATTN_API int cpattn_fwd(const void* q, const void* k, const void* v, void* out
  * 5520-token query slice against a K/V chunk: 352 CTAs are 2.4 waves on 148 SMs, while
  * two key ranges give 704 CTAs.  Same arguments and results as the single-pass calls
  * (bf16 inputs, D in {64, 128}); with n_split = 1 it is exactly that call.
+ * n_split = 0 is the tail split: work items (256 query rows x head x batch, one CTA each)
+ * run over all keys, except the last, partial wave of them -- or that wave and the whole
+ * wave before it -- whose items run as 2..8 key ranges each, as a makespan model of one CTA
+ * per SM chooses (no split when none helps); their fp32 partials are folded afterwards.
+ * n_split larger than the number of 128-key blocks is lowered to it.
  * workspace : caller-owned device buffer, 256-byte aligned, of at least
  *   cpattn_fwd_split_workspace(B, H, Sq, D, n_split, out_dtype) bytes; it receives the
- *   partials ([n_split][B][Sq][H][D] in out_dtype, then [n_split][B][H][Sq] float32).
- *   Concurrent calls must not share it.
- * Errors: as cpattn_fwd / cpattn_fwd_accumulate; CPATTN_ERR_SHAPE for n_split outside 1..8
+ *   partials ([n_split][B][Sq][H][D] in out_dtype, then [n_split][B][H][Sq] float32; for
+ *   n_split = 0, fp32 rows [parts][tail items][256][D], then their float32 LSEs).
+ *   Concurrent calls must not share it.  May be NULL when no partials are needed.
+ * Errors: as cpattn_fwd / cpattn_fwd_accumulate; CPATTN_ERR_SHAPE for n_split outside 0..8
  *   or a workspace that is too small; CPATTN_ERR_ALIGN for its alignment.
  */
 CPATTN_API int cpattn_fwd_split(const void* q, const void* k, const void* v, void* out, float* lse,
@@ -116,7 +122,9 @@ CPATTN_API int cpattn_fwd_split(const void* q, const void* k, const void* v, voi
                                 int accumulate, int n_split, void* workspace,
                                 size_t workspace_bytes, cpattn_stream_t stream);
 
-/* Workspace bytes cpattn_fwd_split needs (0 for n_split = 1 or invalid sizes). */
+/* Workspace bytes cpattn_fwd_split needs (0 for n_split = 1 or invalid sizes).  For
+ * n_split = 0 the plan also depends on the key count, which this query does not take: it
+ * returns the largest workspace any key count can make the call need. */
 CPATTN_API size_t cpattn_fwd_split_workspace(int B, int H, int Sq, int D, int n_split,
                                              int out_dtype);
 
@@ -177,6 +185,31 @@ CPATTN_API size_t cpattn_noalloc_scratch_bytes(void);
 CPATTN_API int cpattn_ulysses_fwd(const void* q, const void* k, const void* v, void* out,
                                   float* lse, int P, int S_local, int H, int D, float scale,
                                   int out_dtype, cpattn_stream_t stream);
+
+/*
+ * cpattn_ulysses_fwd_split -- cpattn_ulysses_fwd with the tail split of cpattn_fwd_split
+ * (n_split = 0): the work items (256 tokens x head, one CTA each; P * ceil(P*S_local/256) *
+ * H/P of them) that fall in the last, partial wave of CTAs -- or in it and the whole wave
+ * before -- run as 2..8 key ranges each, whose fp32 partials (O, LSE) are folded exactly
+ * afterwards (the merge of the Ring Attention step, Fig. 3), so that the GPU's last wave is
+ * short instead of partly idle.  Same arguments and result as cpattn_ulysses_fwd, to
+ * rounding (each range subtracts its own row maximum before P is rounded to bf16, and the
+ * fold runs in fp32), plus:
+ * workspace : caller-owned device buffer, 256-byte aligned, of at least
+ *   cpattn_ulysses_fwd_workspace(P, S_local, H, D, out_dtype) bytes (exact: the key count
+ *   is the query's); NULL allowed when that is 0 (nothing to split: the call is then
+ *   cpattn_ulysses_fwd).  It must not overlap q, k, v, out or lse.
+ * Errors: as cpattn_ulysses_fwd; CPATTN_ERR_NULL / _ALIGN / _SHAPE for a missing,
+ *   misaligned, too small or overlapping workspace.
+ */
+CPATTN_API int cpattn_ulysses_fwd_split(const void* q, const void* k, const void* v, void* out,
+                                        float* lse, int P, int S_local, int H, int D,
+                                        float scale, int out_dtype, void* workspace,
+                                        size_t workspace_bytes, cpattn_stream_t stream);
+
+/* Workspace bytes cpattn_ulysses_fwd_split needs (0: no split, or invalid sizes). */
+CPATTN_API size_t cpattn_ulysses_fwd_workspace(int P, int S_local, int H, int D,
+                                               int out_dtype);
 
 /*
  * cpattn_ulysses_host -- cpattn_ulysses_fwd from host memory to host memory: one whole

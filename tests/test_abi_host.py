@@ -101,6 +101,33 @@ def test_ulysses_fwd_argument_errors(L):
     assert uf(q=FAKE + 8) == B.ERR_ALIGN
 
 
+def test_ulysses_fwd_split_plan_and_argument_errors(L):
+    vp = ctypes.c_void_p
+    # [8][5520][16][128]: 2768 items (8 groups x 2 heads x 173 tile pairs) on 148 SMs leave
+    # 104 in the last wave; the makespan model splits them in 7 key ranges each (728 short
+    # CTAs, 5 short waves of 1/7 of an item): fp32 rows of 7 * 104 * 256, then their LSEs
+    rows = 7 * 104 * 256
+    need = L.cpattn_ulysses_fwd_workspace(8, 5520, 16, 128, 0)
+    assert need == rows * 128 * 4 + rows * 4
+    assert L.cpattn_ulysses_fwd_workspace(8, 5520, 16, 128, 1) == need  # partials are fp32
+    assert L.cpattn_ulysses_fwd_workspace(8, 5520, 16, 96, 0) == 0
+    assert L.cpattn_ulysses_fwd_workspace(8, 5520, 15, 128, 0) == 0  # H % P
+    # one rank of 9472 tokens x 16 heads: 37 tile pairs x 16 = 592 items, 4 whole waves
+    assert L.cpattn_ulysses_fwd_workspace(1, 9472, 16, 128, 0) == 0
+
+    def us(ws=FAKE + (1 << 30), ws_bytes=need, q=FAKE, S_l=5520):
+        return L.cpattn_ulysses_fwd_split(vp(q) if q else None, vp(FAKE), vp(FAKE), vp(FAKE),
+                                          None, 8, S_l, 16, 128, 0.1, 0,
+                                          vp(ws) if ws else None, ws_bytes, None)
+
+    assert us(ws=0) == B.ERR_NULL
+    assert us(ws=FAKE + (1 << 30) + 16) == B.ERR_ALIGN
+    assert us(ws_bytes=need - 1) == B.ERR_SHAPE
+    assert us(ws=FAKE) == B.ERR_SHAPE      # overlaps q (and k, v, out at the same address)
+    assert us(S_l=5512) == B.ERR_UNSUPPORTED  # S_l % 16
+    assert us(q=0) == B.ERR_NULL
+
+
 def test_ulysses_host_argument_errors(L):
     vp = ctypes.c_void_p
     H0, D0 = 0x7000000, 0x100000000  # fake host and device addresses (never dereferenced)
@@ -146,11 +173,16 @@ def test_fwd_split_argument_errors_and_sizes(L):
     assert need == 2 * 512 * 2 * 128 * 2 + 2 * 2 * 512 * 4
     assert L.cpattn_fwd_split_workspace(1, 2, 512, 128, 1, 0) == 0
     assert L.cpattn_fwd_split_workspace(1, 2, 512, 128, 9, 0) == 0
-    # n_split = 0 (tail split) on 148 SMs: 352 items of a [5520][16][128] query leave 56 in
-    # the last wave, each split in 2: fp32 rows of 2 * 56 * 256, then their LSEs
-    rows = 2 * 56 * 256
+    # n_split = 0 (tail split) on 148 SMs: the query does not take the key count, so it
+    # sizes the largest plan: the last wave's items in up to 8 ranges, or those and the
+    # wave before in up to 4.  352 items of a [5520][16][128] query leave 56 in the last
+    # wave: max(56 * 8, (56 + 148) * 4) = 816 tail ranges of 256 fp32 rows, then their LSEs
+    rows = 816 * 256
     assert L.cpattn_fwd_split_workspace(1, 16, 5520, 128, 0, 0) == rows * 128 * 4 + rows * 4
-    assert L.cpattn_fwd_split_workspace(8, 2, 44160, 128, 0, 0) == 0  # 104 left: no room to split
+    # 2768 items of [8][44160][2][128] leave 104: max(104 * 8, 252 * 4) = 1008 ranges
+    rows = 1008 * 256
+    assert L.cpattn_fwd_split_workspace(8, 2, 44160, 128, 0, 0) == rows * 128 * 4 + rows * 4
+    assert L.cpattn_fwd_split_workspace(1, 16, 9472, 128, 0, 0) == 0  # 592 items: 4 whole waves
     assert L.cpattn_fwd_split_workspace(1, 16, 5520, 96, 0, 0) == 0
 
 

@@ -2,8 +2,8 @@
 
 A serving loop records a whole attention step once and replays it; every device call of the
 C ABI is asynchronous on its stream (no allocation, no synchronisation), so the ring step,
-the Ulysses pass through permutes and the fused Ulysses kernel can be captured into a CUDA
-graph.  Each is captured after one eager warm-up, replayed on new inputs copied into the
+the Ulysses pass through permutes and the fused Ulysses kernel (with and without its tail
+split) can be captured into a CUDA graph.  Each is captured after one eager warm-up, replayed on new inputs copied into the
 captured buffers, and compared bit for bit with the same calls run eagerly on those inputs.
 The captured launches keep their programmatic (dependent-launch) edges.
 """
@@ -94,13 +94,21 @@ def test_ulysses_plan_graph_replay(mode):
         assert torch.equal(o_r, o_e) and torch.equal(l_r, l_e), trial
 
 
-def test_fused_ulysses_graph_replay():
-    P, S_l, H, D = 8, 272, 16, 64
+@pytest.mark.parametrize("split", [False, True])
+def test_fused_ulysses_graph_replay(split):
+    # split: 4 groups x 16 heads x 7 tile pairs = 448 items, the last wave's 4 in key ranges
+    P, S_l, H, D = (4, 400, 64, 128) if split else (8, 272, 16, 64)
     shards = [torch.empty(P, S_l, H, D, dtype=torch.bfloat16, device=DEV) for _ in range(3)]
     _refill(shards, 3)
     out = torch.empty(P, S_l, H, D, dtype=torch.bfloat16, device=DEV)
     lse = torch.empty(P, H // P, P * S_l, device=DEV)
-    run = lambda: cp.ulysses_fwd(*shards, P, out=out, lse=lse, scale=1 / math.sqrt(D))
+    if split:
+        ws = torch.empty(cp.ulysses_workspace_bytes(P, S_l, H, D), dtype=torch.uint8, device=DEV)
+        assert ws.numel() > 0
+        run = lambda: cp.ulysses_fwd_split(*shards, P, out=out, lse=lse, scale=1 / math.sqrt(D),
+                                           workspace=ws)
+    else:
+        run = lambda: cp.ulysses_fwd(*shards, P, out=out, lse=lse, scale=1 / math.sqrt(D))
     graph, _ = _capture(run)
     for trial in range(2):
         _refill(shards, 300 + trial)

@@ -101,6 +101,21 @@ def test_guard_bands_fused_ulysses(P, S_l, H, D, out_dtype):
     _check(o, l)
 
 
+@pytest.mark.parametrize("P,S_l,H,D", [(4, 400, 64, 128), (3, 336, 24, 64)])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_guard_bands_fused_ulysses_tail_split(P, S_l, H, D, out_dtype):
+    g = torch.Generator().manual_seed(P * 11 + S_l)
+    shards = [W.randn((P, S_l, H, D), g, 1.0, "bf16").to(DEV) for _ in range(3)]
+    need = cp.ulysses_workspace_bytes(P, S_l, H, D, out_dtype)
+    assert need > 0
+    o = Guarded((P, S_l, H, D), out_dtype)
+    l = Guarded((P, H // P, P * S_l), torch.float32)
+    wbuf = torch.full((need + 2 * GUARD_BYTES,), 0xA5, dtype=torch.uint8, device=DEV)
+    cp.ulysses_fwd_split(*shards, P, out=o.t, lse=l.t, workspace=wbuf[GUARD_BYTES:GUARD_BYTES + need])
+    _check(o, l)
+    assert bool((wbuf[:GUARD_BYTES] == 0xA5).all()) and bool((wbuf[GUARD_BYTES + need:] == 0xA5).all())
+
+
 @pytest.mark.parametrize("Bn,S,H,D,dt", [(1, 301, 3, 128, torch.bfloat16), (2, 77, 2, 64, torch.float32),
                                          (1, 5, 1, 1024, torch.float32)])
 def test_guard_bands_merge(Bn, S, H, D, dt):

@@ -481,6 +481,62 @@ def test_fused_ulysses_full_size_bit_identical():
     assert torch.equal(out_f, out_u) and torch.equal(lse_f, lse_u)
 
 
+# Fused Ulysses with the tail split.  (4, 400, 64): 448 items (4 groups x 16 heads x 7 tile
+# pairs) on 148 SMs leave 4, split in 6 key ranges; (8, 1040, 16): 528 items (8 x 2 x 33)
+# leave 84, split in 5; (3, 336, 24, 64): 96 items in 3 ranges each, ragged last tile pairs.
+@pytest.mark.parametrize("P,S_l,H,D", [(4, 400, 64, 128), (8, 1040, 16, 128), (3, 336, 24, 64)])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_fused_ulysses_tail_split_matches_oracle(P, S_l, H, D, out_dtype):
+    need = cp.ulysses_workspace_bytes(P, S_l, H, D, out_dtype)
+    assert need > 0, "the shape must exercise the split"
+    g = torch.Generator().manual_seed(P * 7 + S_l + H)
+    shards = [W.randn((P, S_l, H, D), g, 1.0, "bf16").to(DEV) for _ in range(3)]
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device=DEV)  # garbage in the workspace
+    out_t, lse_t = cp.ulysses_fwd_split(*shards, P, out_dtype=out_dtype, workspace=ws)
+    out_1, lse_1 = cp.ulysses_fwd(*shards, P, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    full = lambda t: t.cpu().reshape(1, P * S_l, H, D)
+    rows = W.sample_rows(1, H, P * S_l, 2048, seed=P + S_l)
+    o_ref, l_ref = ref.attention_rows(full(shards[0]), full(shards[1]), full(shards[2]),
+                                      1 / math.sqrt(D), rows)
+    oc = out_t.cpu().reshape(1, P * S_l, H, D)
+    lc = lse_t.cpu().reshape(1, H, P * S_l)
+    kind = "bf16_out" if out_dtype == torch.bfloat16 else "bf16_in"
+    check_o(torch.stack([oc[b, i, h] for (b, h, i) in rows]), o_ref, kind, f"split {P},{S_l},{H}")
+    check_lse(torch.stack([lc[b, h, i] for (b, h, i) in rows]), l_ref, f"split {P},{S_l},{H}")
+    # the unsplit kernel on the same shards: equal to rounding (each key range subtracts its
+    # own row maximum before P is rounded to bf16; the fold runs in fp32)
+    assert (lse_t - lse_1).abs().max().item() < 2e-5
+    tol = 2e-3 if out_dtype == torch.float32 else 1e-2
+    assert (out_t.float() - out_1.float()).abs().max().item() < tol
+    # relative L2 of the difference: the two sides round P to bf16 against different row
+    # maxima, so each carries its own P rounding noise (about 2^-9 per weight; measured
+    # 1.2-1.8e-3 here), and bf16 outputs add their own rounding
+    assert rel_l2(out_t, out_1) < 5e-3
+
+
+def test_fused_ulysses_tail_split_full_size():
+    # the bench workload: 2768 items, the last wave's 104 split in 7 key ranges
+    w = W.WORKLOADS[4]
+    x = W.make_inputs(w)
+    P = w.P
+    q, k, v = (x[n].to(DEV) for n in ("q", "k", "v"))
+    out_t, lse_t = cp.ulysses_fwd_split(q, k, v, P)
+    out_1, lse_1 = cp.ulysses_fwd(q, k, v, P)
+    torch.cuda.synchronize()
+    assert (lse_t - lse_1).abs().max().item() < 2e-5
+    assert (out_t.float() - out_1.float()).abs().max().item() < 1e-2
+    # sampled rows of the split items against the oracle (the last 104 items: group 7)
+    S_l, H = q.shape[1], q.shape[2]
+    full = lambda t: t.cpu().reshape(1, P * S_l, H, w.D)
+    rows = W.sample_rows(1, H, P * S_l, 1024, seed=17)
+    o_ref, l_ref = ref.attention_rows(full(q), full(k), full(v), w.softmax_scale, rows)
+    oc = out_t.cpu().reshape(1, P * S_l, H, w.D)
+    lc = lse_t.cpu().reshape(1, H, P * S_l)
+    check_o(torch.stack([oc[b, i, h] for (b, h, i) in rows]), o_ref, "bf16_out", "split full")
+    check_lse(torch.stack([lc[b, h, i] for (b, h, i) in rows]), l_ref, "split full")
+
+
 # ----------------------------------------------------------------------------- host-buffer pass
 
 
