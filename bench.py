@@ -49,12 +49,12 @@ ATTN_SOURCES = ("context_long_sequence_non_b200/csrc/attn_sm100.cu",
                 "context_long_sequence_non_b200/csrc/sm100_ptx.cuh")
 ATTN_TRAFFIC = {
     "attn_fwd_sm100_kernel<128,0,2>": {  # the fused Ulysses kernel, one launch per step
-        "sources_sha256": "ea5b7c0fb489155c8ff3494afb99ffc8aca83f3006d1b33331772d07d17431f0",
-        "bytes": 594_595_584 + 169_908_224,
+        "sources_sha256": "362e6b2520cec910859994b7e7a27fdade9dbc362535f505f9df498f6af2791e",
+        "bytes": 575_498_752 + 167_627_776,
     },
     "attn_fwd_sm100_kernel<128,0,0>": {  # the plain form, in the 5-launch step
-        "sources_sha256": "ea5b7c0fb489155c8ff3494afb99ffc8aca83f3006d1b33331772d07d17431f0",
-        "bytes": 571_694_592 + 168_004_608,
+        "sources_sha256": "362e6b2520cec910859994b7e7a27fdade9dbc362535f505f9df498f6af2791e",
+        "bytes": 566_098_688 + 167_009_280,
     },
 }
 AUX_REPS = 15  # bursts per auxiliary measurement (median reported, with the range)
