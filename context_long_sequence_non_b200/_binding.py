@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
                                            ctypes.c_size_t, vp]
             L.cpattn_fwd_split_workspace.argtypes = [i, i, i, i, i, i]
             L.cpattn_fwd_split_workspace.restype = ctypes.c_size_t
+            L.cpattn_fwd_split_workspace_kv.argtypes = [i, i, i, i, i, i, i]
+            L.cpattn_fwd_split_workspace_kv.restype = ctypes.c_size_t
             L.cpattn_split_suggest.argtypes = [i, i, i, i]
             L.cpattn_merge.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
             L.cpattn_seq2head.argtypes = [vp, vp, i, i, i, i, i, vp]
@@ -227,7 +229,12 @@ def ulysses_host(hq, hk, hv, h_out, h_lse, dq, dk, dv, d_out, d_lse, P, scale=No
     return h_out, h_lse
 
 
-def split_workspace_bytes(B, H, Sq, D, n_split, out_dtype=torch.bfloat16) -> int:
+def split_workspace_bytes(B, H, Sq, D, n_split, out_dtype=torch.bfloat16, Skv=None) -> int:
+    """Workspace bytes of fwd_split: exact for the key count ``Skv`` when given, else (for
+    the tail split, n_split = 0) the largest any key count can need."""
+    if Skv is not None:
+        return int(lib().cpattn_fwd_split_workspace_kv(B, H, Sq, Skv, D, n_split,
+                                                       _dtype_code(out_dtype)))
     return int(lib().cpattn_fwd_split_workspace(B, H, Sq, D, n_split, _dtype_code(out_dtype)))
 
 
@@ -251,7 +258,7 @@ def fwd_split(q, k, v, out=None, lse=None, scale=None, out_dtype=None, accumulat
         lse = torch.empty((B_, H, Sq), dtype=torch.float32, device=q.device)
     if n_split is None:
         n_split = split_suggest(B_, H, Sq, Skv)
-    need = split_workspace_bytes(B_, H, Sq, D, n_split, out.dtype)
+    need = split_workspace_bytes(B_, H, Sq, D, n_split, out.dtype, Skv=Skv)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
     _need_cuda(q, k, v, out, lse, workspace)

@@ -190,6 +190,21 @@ size_t cpattn_fwd_split_workspace(int B, int H, int Sq, int D, int n_split, int 
   return n_split == 1 ? 0 : split_ws_bytes(B, H, Sq, D, n_split, es);
 }
 
+size_t cpattn_fwd_split_workspace_kv(int B, int H, int Sq, int Skv, int D, int n_split,
+                                     int out_dtype) {
+  const int es = elem_size(out_dtype);
+  if (B < 1 || H < 1 || Sq < 1 || Skv < 1 || D < 1 || n_split < 0 || n_split > kMaxSplit ||
+      es == 0)
+    return 0;
+  if (n_split == 0) {
+    if (D != 64 && D != 128) return 0;
+    return cpattn::tail_split_workspace(cpattn::tail_split_plan(B, H, Sq, Skv), D);
+  }
+  const int n_kv = (Skv + 127) / 128;
+  const int n = n_split > n_kv ? n_kv : n_split;  // the lowering cpattn_fwd_split applies
+  return n <= 1 ? 0 : split_ws_bytes(B, H, Sq, D, n, es);
+}
+
 int cpattn_split_suggest(int B, int H, int Sq, int Skv) {
   if (B < 1 || H < 1 || Sq < 1 || Skv < 1) return 1;
   const long long ctas = (long long)((Sq + 255) / 256) * H * B;

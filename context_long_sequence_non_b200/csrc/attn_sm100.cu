@@ -717,11 +717,12 @@ TailSplit tail_split_plan(int B, int H, int Sq, int Skv) {
   if (items < 1 || items > 0x7fffffffLL || n_kv < 4) return t;
   const long long rem = items % sms;  // items of the last, partial wave
   if (rem == 0) return t;
-  // Makespan in units of one whole item's time, each CTA paying a fixed start-up and
-  // epilogue of about two key blocks (c): whole waves cost 1 + c, and the split items'
-  // ranges run in ceil(tail * p / sms) short waves of 1/p + c.  Split only when that saves
-  // at least 0.5 %.
-  const double c = 2.0 / n_kv;
+  // Makespan in units of one whole item's time, each CTA paying a fixed cost (c) of about
+  // eight key blocks -- start-up, Q load, pipeline fill, epilogue and its share of the
+  // combine; calibrated on measured splits of short and long items: whole waves cost 1 + c,
+  // and the split items' ranges run in ceil(tail * p / sms) short waves of 1/p + c.  Split
+  // only when that saves at least 0.5 %.
+  const double c = 8.0 / n_kv;
   const double whole = double((items + sms - 1) / sms) * (1.0 + c);
   double best = whole * 0.995;
   for (int k = 0; k < 2; ++k) {

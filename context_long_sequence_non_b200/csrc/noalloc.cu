@@ -66,12 +66,9 @@ int cpattn_fwd_split_noalloc(const void* q, const void* k, const void* v, void* 
   // the split count cpattn_fwd_split will actually use: that call lowers n_split to the
   // number of 128-key blocks (every range holds at least one), so a request such as
   // n_split = 8 over 256 keys needs the scratch of two ranges, not eight.
-  int n_used = n_split;
-  if (n_split >= 1 && Skv >= 0) {
-    const int n_kv = (Skv + 127) / 128;
-    if (n_used > n_kv) n_used = n_kv > 0 ? n_kv : 1;
-  }
-  if (cpattn_fwd_split_workspace(B, H, Sq, D, n_used, out_dtype) > kNoAllocScratchBytes)
+  // For the tail split (n_split = 0) it is made for this call's own plan, which depends on
+  // the key count: cpattn_fwd_split_workspace_kv gives the exact need either way.
+  if (cpattn_fwd_split_workspace_kv(B, H, Sq, Skv, D, n_split, out_dtype) > kNoAllocScratchBytes)
     return CPATTN_ERR_SHAPE;
   int status = CPATTN_OK;
   void* scratch = scratch_on_current_device(&status);

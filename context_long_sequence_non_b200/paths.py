@@ -42,8 +42,9 @@ def ring_attention(q, k_chunks, v_chunks, scale=None, acc_dtype=None, fused=True
         if n_split is None:
             n_split = B.split_suggest(Bn, H, Sq, k_chunks[0].shape[1])
         if n_split != 1:
-            ws = torch.empty(max(B.split_workspace_bytes(Bn, H, Sq, D, n_split, acc_dtype), 256),
-                             dtype=torch.uint8, device=q.device)
+            need = max(B.split_workspace_bytes(Bn, H, Sq, D, n_split, acc_dtype, Skv=kc.shape[1])
+                       for kc in k_chunks)
+            ws = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
             acc_l.fill_(-math.inf)  # empty accumulator: its O rows are never read
             for kc, vc in zip(k_chunks, v_chunks):
                 B.fwd_split(q, kc, vc, out=acc_o, lse=acc_l, scale=scale, accumulate=True,

@@ -128,6 +128,12 @@ CPATTN_API int cpattn_fwd_split(const void* q, const void* k, const void* v, voi
 CPATTN_API size_t cpattn_fwd_split_workspace(int B, int H, int Sq, int D, int n_split,
                                              int out_dtype);
 
+/* Workspace bytes cpattn_fwd_split needs for this key count: exact, for every n_split
+ * (after the call's lowering of n_split to the number of 128-key blocks); 0 when nothing
+ * is split or the sizes are invalid. */
+CPATTN_API size_t cpattn_fwd_split_workspace_kv(int B, int H, int Sq, int Skv, int D,
+                                                int n_split, int out_dtype);
+
 /*
  * cpattn_split_suggest -- split count (1..8) the library's wave model prefers for this
  * shape on the current device: 1 when the (query tile pair, head) grid already fills the
@@ -158,8 +164,8 @@ CPATTN_API int cpattn_split_suggest(int B, int H, int Sq, int Skv);
  * the GPU -- on different streams, or from different threads -- race on it and must not
  * be issued.
  * Errors: as cpattn_fwd_split; CPATTN_ERR_SHAPE also when the partials need more than
- *   cpattn_noalloc_scratch_bytes() (cpattn_fwd_split_workspace(B, H, Sq, D, n_split,
- *   out_dtype) tells), checked before anything is launched.
+ *   cpattn_noalloc_scratch_bytes() (cpattn_fwd_split_workspace_kv(B, H, Sq, Skv, D,
+ *   n_split, out_dtype) tells), checked before anything is launched.
  */
 CPATTN_API int cpattn_fwd_split_noalloc(const void* q, const void* k, const void* v, void* out,
                                         float* lse, int B, int H, int Sq, int Skv, int D,

@@ -104,9 +104,9 @@ def test_ulysses_fwd_argument_errors(L):
 def test_ulysses_fwd_split_plan_and_argument_errors(L):
     vp = ctypes.c_void_p
     # [8][5520][16][128]: 2768 items (8 groups x 2 heads x 173 tile pairs) on 148 SMs leave
-    # 104 in the last wave; the makespan model splits them in 7 key ranges each (728 short
-    # CTAs, 5 short waves of 1/7 of an item): fp32 rows of 7 * 104 * 256, then their LSEs
-    rows = 7 * 104 * 256
+    # 104 in the last wave; the makespan model splits them in 4 key ranges each (416 short
+    # CTAs, 3 short waves of 1/4 of an item): fp32 rows of 4 * 104 * 256, then their LSEs
+    rows = 4 * 104 * 256
     need = L.cpattn_ulysses_fwd_workspace(8, 5520, 16, 128, 0)
     assert need == rows * 128 * 4 + rows * 4
     assert L.cpattn_ulysses_fwd_workspace(8, 5520, 16, 128, 1) == need  # partials are fp32
@@ -184,6 +184,19 @@ def test_fwd_split_argument_errors_and_sizes(L):
     assert L.cpattn_fwd_split_workspace(8, 2, 44160, 128, 0, 0) == rows * 128 * 4 + rows * 4
     assert L.cpattn_fwd_split_workspace(1, 16, 9472, 128, 0, 0) == 0  # 592 items: 4 whole waves
     assert L.cpattn_fwd_split_workspace(1, 16, 5520, 96, 0, 0) == 0
+    # exact sizes for a key count: the ring chunk (5520 keys) splits its 56 items in 2 (one
+    # short wave); the [8][44160][2][128] pass splits the last wave's 104 items in 4
+    kv = L.cpattn_fwd_split_workspace_kv
+    rows = 2 * 56 * 256
+    assert kv(1, 16, 5520, 5520, 128, 0, 0) == rows * 128 * 4 + rows * 4
+    rows = 4 * 104 * 256
+    assert kv(8, 2, 44160, 44160, 128, 0, 0) == rows * 128 * 4 + rows * 4
+    assert kv(1, 20, 3000, 3000, 128, 0, 0) == 0  # 24 key blocks: short ranges do not pay
+    assert kv(1, 16, 5520, 300, 128, 0, 0) == 0  # 3 key blocks: ranges of 2 do not pay
+    # split-KV: lowered to the key blocks there are, as the call lowers it
+    assert kv(1, 8, 4096, 256, 128, 8, 0) == L.cpattn_fwd_split_workspace(1, 8, 4096, 128, 2, 0)
+    assert kv(1, 8, 4096, 100, 128, 8, 0) == 0  # one key block: nothing to split
+    assert kv(1, 2, 512, 0, 128, 2, 0) == 0
 
 
 def test_split_suggestion_model():

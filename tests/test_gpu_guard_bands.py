@@ -101,7 +101,7 @@ def test_guard_bands_fused_ulysses(P, S_l, H, D, out_dtype):
     _check(o, l)
 
 
-@pytest.mark.parametrize("P,S_l,H,D", [(4, 400, 64, 128), (3, 336, 24, 64)])
+@pytest.mark.parametrize("P,S_l,H,D", [(4, 400, 64, 128), (3, 688, 24, 64)])
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
 def test_guard_bands_fused_ulysses_tail_split(P, S_l, H, D, out_dtype):
     g = torch.Generator().manual_seed(P * 11 + S_l)

@@ -38,6 +38,8 @@ def lib():
     L.cpattn_fwd_split.restype = i
     L.cpattn_fwd_split_workspace.argtypes = [i, i, i, i, i, i]
     L.cpattn_fwd_split_workspace.restype = ctypes.c_size_t
+    L.cpattn_fwd_split_workspace_kv.argtypes = [i, i, i, i, i, i, i]
+    L.cpattn_fwd_split_workspace_kv.restype = ctypes.c_size_t
     L.cpattn_noalloc_scratch_bytes.argtypes = []
     L.cpattn_noalloc_scratch_bytes.restype = ctypes.c_size_t
     L.cpattn_device_error.argtypes = []
@@ -73,8 +75,9 @@ def test_noalloc_matches_workspace_entry_point(lib, case, out_dtype):
     k2, v2 = (torch.randn(B, Skv, H, D, generator=g).to(torch.bfloat16).cuda() for _ in range(2))
     scale = 1.0 / math.sqrt(D)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    need = lib.cpattn_fwd_split_workspace(B, H, Sq, D, n_used, dt)
+    need = lib.cpattn_fwd_split_workspace_kv(B, H, Sq, Skv, D, n_split, dt)  # exact
     assert 0 < need <= lib.cpattn_noalloc_scratch_bytes()
+    assert need == lib.cpattn_fwd_split_workspace_kv(B, H, Sq, Skv, D, n_used, dt)
     if n_used != n_split:  # the unlowered request alone would not fit
         assert lib.cpattn_fwd_split_workspace(B, H, Sq, D, n_split, dt) > \
             lib.cpattn_noalloc_scratch_bytes()
