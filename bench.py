@@ -49,12 +49,12 @@ ATTN_SOURCES = ("context_long_sequence_non_b200/csrc/attn_sm100.cu",
                 "context_long_sequence_non_b200/csrc/sm100_ptx.cuh")
 ATTN_TRAFFIC = {
     "attn_fwd_sm100_kernel<128,0,2>": {  # the fused Ulysses kernel, one launch per step
-        "sources_sha256": "362e6b2520cec910859994b7e7a27fdade9dbc362535f505f9df498f6af2791e",
-        "bytes": 575_498_752 + 167_627_776,
+        "sources_sha256": "f378744a573de89c4ef13c37cdd112e213b64b4a9cd4b6ebd0c092bfc867aa61",
+        "bytes": 577_045_504 + 167_678_720,
     },
     "attn_fwd_sm100_kernel<128,0,0>": {  # the plain form, in the 5-launch step
-        "sources_sha256": "362e6b2520cec910859994b7e7a27fdade9dbc362535f505f9df498f6af2791e",
-        "bytes": 566_098_688 + 167_009_280,
+        "sources_sha256": "f378744a573de89c4ef13c37cdd112e213b64b4a9cd4b6ebd0c092bfc867aa61",
+        "bytes": 584_850_688 + 168_275_200,
     },
 }
 AUX_REPS = 15  # bursts per auxiliary measurement (median reported, with the range)
