@@ -30,7 +30,8 @@ def ring_attention(q, k_chunks, v_chunks, scale=None, acc_dtype=None, fused=True
     form, ``n_split`` > 1 (or None: the library's suggestion) computes every chunk as that
     many key ranges folded straight into the accumulator (split-KV, for query slices too
     small to fill the GPU), and ``n_split = 0`` splits only the work items of each chunk's
-    last, partial wave of CTAs (tail split).  Returns ``(O, LSE)``.
+    last wave or two of CTAs, as the library's makespan model chooses (tail split).
+    Returns ``(O, LSE)``.
     """
     if scale is None:
         scale = 1.0 / math.sqrt(q.shape[3])
