@@ -297,3 +297,23 @@ def test_product_path_has_no_oracle_or_fallback():
                 with open(os.path.join(dirpath, fn)) as f:
                     src = f.read()
                 assert "import oracle" not in src and "from oracle" not in src, fn
+
+
+def test_tail_split_workspace_bound_holds_for_every_key_count(L):
+    # the n_split = 0 query takes no key count and promises an upper bound: the exact need
+    # of every key count stays below it (a caller sizing by the bound never runs short)
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+
+    @settings(max_examples=300, deadline=None)
+    @given(st.integers(1, 8), st.integers(1, 64), st.integers(1, 60000), st.integers(1, 60000),
+           st.sampled_from([64, 128]), st.sampled_from([0, 1]))
+    def check(Bn, H, Sq, Skv, D, dt):
+        exact = L.cpattn_fwd_split_workspace_kv(Bn, H, Sq, Skv, D, 0, dt)
+        bound = L.cpattn_fwd_split_workspace(Bn, H, Sq, D, 0, dt)
+        assert exact <= bound
+        if exact:  # fp32 rows of 256 per range, then their LSEs
+            rows = exact // (D * 4 + 4)
+            assert rows % 256 == 0 and exact == rows * D * 4 + rows * 4
+
+    check()
