@@ -317,3 +317,18 @@ def test_tail_split_workspace_bound_holds_for_every_key_count(L):
             assert rows % 256 == 0 and exact == rows * D * 4 + rows * 4
 
     check()
+
+
+def test_ulysses_workspace_is_the_plain_plan_of_its_head_groups(L):
+    # the fused pass splits the same work items as a [P][P*S_l][H/P][D] attention would
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+
+    @settings(max_examples=200, deadline=None)
+    @given(st.integers(1, 8), st.integers(1, 600), st.integers(1, 8), st.sampled_from([64, 128]))
+    def check(P, s16, hp, D):
+        S_l, H = 16 * s16, hp * P
+        assert L.cpattn_ulysses_fwd_workspace(P, S_l, H, D, 0) == \
+            L.cpattn_fwd_split_workspace_kv(P, hp, P * S_l, P * S_l, D, 0, 0)
+
+    check()
