@@ -526,6 +526,28 @@ def next_paths(cp, w, q, k, v, plan, dev, stream):
         return statistics.median(ts)
 
     res = {}
+    # the bandwidth kernels first, right after the idle, before the attention entries heat
+    # the GPU into its power cap (their issue-bound forms follow the SM clock)
+    ms = timed(lambda: cp.seq2head_qkv(q, k, v, w.P, out=(plan.qh, plan.kh, plan.vh)))
+    nbytes = 3 * 2 * q.numel() * q.element_size()
+    res["seq2head_qkv"] = {"ms": round(ms, 4), "bytes": nbytes,
+                           "GB/s": round(nbytes / ms / 1e6, 1),
+                           "frac_of_hbm": round(nbytes / ms / 1e6 / peaks["hbm_gbs"], 4)}
+    # the sample's Q/K RMSNorm fused into that launch (same bytes), and standalone in place
+    gq = W.norm_weights(w.D, seed=41).to(dev)
+    gk = W.norm_weights(w.D, seed=42).to(dev)
+    ms = timed(lambda: cp.seq2head_qkv_norm(q, k, v, w.P, gq, gk, out=(plan.qh, plan.kh, plan.vh)))
+    res["seq2head_qkv_norm"] = {"ms": round(ms, 4), "bytes": nbytes,
+                                "GB/s": round(nbytes / ms / 1e6, 1),
+                                "frac_of_hbm": round(nbytes / ms / 1e6 / peaks["hbm_gbs"], 4),
+                                "what": "seq2head of Q, K, V with RMSNorm of Q and K head rows"}
+    qn = q.clone()
+    nb1 = 2 * qn.numel() * qn.element_size()
+    ms = timed(lambda: cp.rmsnorm(qn, gq, out=qn))
+    res["rmsnorm"] = {"ms": round(ms, 4), "bytes": nb1, "GB/s": round(nb1 / ms / 1e6, 1),
+                      "frac_of_hbm": round(nb1 / ms / 1e6 / peaks["hbm_gbs"], 4),
+                      "what": "RMSNorm of [8][5520][16][128] bf16 head rows, in place"}
+    del qn
     # the image-DiT joint sequence: B=1, H=24, S=4608 (4096 image + 512 text tokens), D=128
     w2 = W.WORKLOADS[2]
     x2 = W.make_inputs(w2)
@@ -558,26 +580,6 @@ def next_paths(cp, w, q, k, v, plan, dev, stream):
     res["ulysses_fused_split"] = {"ms": round(ms, 4), "TFLOP/s": round(w.attn_flops / ms / 1e9, 2),
                                   "what": "the same with the tail split (cpattn_ulysses_fwd_split)"}
     del ws_u
-    ms = timed(lambda: cp.seq2head_qkv(q, k, v, w.P, out=(plan.qh, plan.kh, plan.vh)))
-    nbytes = 3 * 2 * q.numel() * q.element_size()
-    res["seq2head_qkv"] = {"ms": round(ms, 4), "bytes": nbytes,
-                           "GB/s": round(nbytes / ms / 1e6, 1),
-                           "frac_of_hbm": round(nbytes / ms / 1e6 / peaks["hbm_gbs"], 4)}
-    # the sample's Q/K RMSNorm fused into that launch (same bytes), and standalone in place
-    gq = W.norm_weights(w.D, seed=41).to(dev)
-    gk = W.norm_weights(w.D, seed=42).to(dev)
-    ms = timed(lambda: cp.seq2head_qkv_norm(q, k, v, w.P, gq, gk, out=(plan.qh, plan.kh, plan.vh)))
-    res["seq2head_qkv_norm"] = {"ms": round(ms, 4), "bytes": nbytes,
-                                "GB/s": round(nbytes / ms / 1e6, 1),
-                                "frac_of_hbm": round(nbytes / ms / 1e6 / peaks["hbm_gbs"], 4),
-                                "what": "seq2head of Q, K, V with RMSNorm of Q and K head rows"}
-    qn = q.clone()
-    nb1 = 2 * qn.numel() * qn.element_size()
-    ms = timed(lambda: cp.rmsnorm(qn, gq, out=qn))
-    res["rmsnorm"] = {"ms": round(ms, 4), "bytes": nb1, "GB/s": round(nb1 / ms / 1e6, 1),
-                      "frac_of_hbm": round(nb1 / ms / 1e6 / peaks["hbm_gbs"], 4),
-                      "what": "RMSNorm of [8][5520][16][128] bf16 head rows, in place"}
-    del qn
     w3 = W.WORKLOADS[3]
     x3 = W.make_inputs(w3)
     q3, k3, v3 = (x3[n].to(dev) for n in ("q", "k", "v"))
