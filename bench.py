@@ -2,13 +2,17 @@
 """Benchmark of the per-rank context-parallel attention hot path on B200.
 
 One step = one pass of the Ulysses path over the S=44160 video-latent workload:
-P=8 virtual ranks x [5520 tokens][16 heads][128] bf16 Q/K/V -> 3 seq2head permutes ->
-non-causal attention over B=8 head groups x 2 heads x S=44160 x D=128 (tcgen05 kernel)
--> head2seq permute.  The metric is attention TFLOPS (4*B*H*S^2*D per step) over the
-whole step; the attention kernel's own roofline, the permutes' and the (O, LSE) merge's
-HBM rooflines and an end-to-end number through host buffers are reported beside it.
+P=8 virtual ranks x [5520 tokens][16 heads][128] bf16 Q/K/V shards in, non-causal
+attention over 8 head groups x 2 heads x S=44160 x D=128, O shards + LSE out.  Two step
+variants of the same work are timed: `fused` (the default headline: one tcgen05 kernel
+whose addressing does the re-partitions) and `plain` (3 seq2head permutes -> attention ->
+head2seq).  The metric is attention TFLOPS (4*B*H*S^2*D per step) over the whole step;
+the attention kernel's own roofline, the permutes' and the (O, LSE) merge's HBM rooflines,
+the other workloads' attention and an end-to-end number through host buffers are
+reported beside it.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--step fused|plain] [--qk-norm] [--profile] [--no-cpu-baseline]
 
 Under torchrun (N > 1) every rank runs its own replica (weak scaling, no data-path
 collective); the timed region is bracketed by barriers and the max over ranks is used.
