@@ -823,6 +823,59 @@ def cpu_baseline(budget_s=15.0):
             "kind": "oracle", "sample": _sample_text(rounds * ORACLE_ROWS, spent)}
 
 
+def oracle_per_config(row_sample=2048):
+    """The fp64 oracle timed on each configuration's own inputs on the host cores (one JSON
+    line).  Configs 1 and 2 run in full; config 3 as one of its eight K/V chunks plus one
+    merge, scaled to the eight chunks and seven merges; configs 4 and 5 on ``row_sample``
+    sampled query rows, scaled to all rows.  Each entry says which."""
+    import oracle
+
+    cores = oracle.set_threads()
+    out = {"kind": "oracle", "cores": cores, "configs": {}}
+    for n, w in W.WORKLOADS.items():
+        x = W.make_inputs(w)
+        flops = w.attn_flops
+        if w.kind == "chunked":  # fp32, two chunks folded by the merge
+            t = time.perf_counter()
+            c = x["chunks"][0]
+            oa, la = oracle.attention(x["q"], x["k"][:, :c], x["v"][:, :c], w.softmax_scale)
+            ob, lb = oracle.attention(x["q"], x["k"][:, c:], x["v"][:, c:], w.softmax_scale)
+            oracle.merge(oa, la, ob, lb)
+            sec, how = time.perf_counter() - t, "full: two chunks and their merge"
+        elif w.kind == "single" and flops < 1e12:
+            t = time.perf_counter()
+            oracle.attention(x["q"], x["k"], x["v"], w.softmax_scale)
+            sec, how = time.perf_counter() - t, "full"
+        elif w.kind == "ring":
+            c = x["chunks"][0]
+            t = time.perf_counter()
+            oa, la = oracle.attention(x["q"], x["k"][:, :c], x["v"][:, :c], w.softmax_scale)
+            t1 = time.perf_counter()
+            oracle.merge(oa, la, oa, la)
+            t2 = time.perf_counter()
+            sec = 8 * (t1 - t) + 7 * (t2 - t1)
+            how = "one of the 8 chunks and one merge, timed and scaled to 8 chunks + 7 merges"
+        else:  # the long sequences (Ulysses, joint video + text): sampled rows, all keys
+            S = w.Sq
+            H = w.H * w.P if w.kind == "ulysses" else w.H
+            full = (lambda t: t.reshape(1, S, H, w.D)) if w.kind == "ulysses" else (lambda t: t)
+            g = torch.Generator(device="cpu").manual_seed(500 + n)
+            hs = torch.randint(0, H, (row_sample,), generator=g).tolist()
+            ts = torch.randint(0, S, (row_sample,), generator=g).tolist()
+            rows = [(0, h, i) for h, i in zip(hs, ts)]
+            oracle.attention_rows(full(x["q"]), full(x["k"]), full(x["v"]), w.softmax_scale,
+                                  rows[: row_sample // 8])  # untimed: page-in, BLAS threads
+            t = time.perf_counter()
+            oracle.attention_rows(full(x["q"]), full(x["k"]), full(x["v"]), w.softmax_scale, rows)
+            dt = time.perf_counter() - t
+            sec = dt * (H * S) / row_sample
+            how = f"{row_sample} sampled query rows over all {S} keys, scaled to all {H * S} rows"
+        out["configs"][w.name] = {"seconds": round(sec, 3), "flops": flops,
+                                  "TFLOP/s": round(flops / sec / 1e12, 6), "how": how}
+        del x
+    return out
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return  # the CPU oracle arm runs on rank 0 only
@@ -857,6 +910,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--oracle-configs", action="store_true",
+                    help="time the CPU oracle on every configuration (host only) and exit")
     ap.add_argument("--profile", action="store_true",
                     help="for profiler captures: run only warm-up + timed steps (no aux "
                          "kernels, no end-to-end pass, no CPU baseline)")
@@ -874,6 +929,10 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
     world, rank, local = dist_env()
+    if args.oracle_configs:  # the oracle's own timing table (host cores only, no GPU work)
+        if rank == 0:
+            print(json.dumps(oracle_per_config()), flush=True)
+        return
     if args.impl == "reference":
         run_reference(args, world, rank)
     else:
