@@ -121,6 +121,21 @@ def _need_cuda(*ts):
                 raise ValueError("tensors must be contiguous")
 
 
+def _need_shape(t, shape, name, dtype=None):
+    """A caller-provided output must have exactly the size the call writes: the library
+    receives only its pointer."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, not {tuple(t.shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, not {t.dtype}")
+
+
+def _nbytes(t):
+    return 0 if t is None else t.numel() * t.element_size()
+
+
 def fwd(q, k, v, out=None, lse=None, scale=None, out_dtype=None, want_lse=True, stream=None):
     """Non-causal attention ``softmax(scale * Q K^T) V`` with its log-sum-exp.
 
@@ -139,6 +154,8 @@ def fwd(q, k, v, out=None, lse=None, scale=None, out_dtype=None, want_lse=True, 
         out = torch.empty((B, Sq, H, D), dtype=out_dtype, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    _need_shape(out, (B, Sq, H, D), "out")
+    _need_shape(lse, (B, H, Sq), "lse", torch.float32)
     _need_cuda(q, k, v, out, lse)
     st = lib().cpattn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Sq, Skv, D,
                           float(scale), _dtype_code(q.dtype), _dtype_code(out.dtype),
@@ -160,6 +177,8 @@ def ulysses_fwd(q, k, v, P, out=None, lse=None, scale=None, out_dtype=None, want
         out = torch.empty((P, S_l, H, D), dtype=out_dtype or q.dtype, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((P, H // P, P * S_l), dtype=torch.float32, device=q.device)
+    _need_shape(out, (P, S_l, H, D), "out")
+    _need_shape(lse, (P, H // P, P * S_l), "lse", torch.float32)
     _need_cuda(q, k, v, out, lse)
     st = lib().cpattn_ulysses_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), P, S_l, H, D,
                                   float(scale), _dtype_code(out.dtype), _stream(stream))
@@ -186,15 +205,15 @@ def ulysses_fwd_split(q, k, v, P, out=None, lse=None, scale=None, out_dtype=None
         out = torch.empty((P, S_l, H, D), dtype=out_dtype or q.dtype, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((P, H // P, P * S_l), dtype=torch.float32, device=q.device)
+    _need_shape(out, (P, S_l, H, D), "out")
+    _need_shape(lse, (P, H // P, P * S_l), "lse", torch.float32)
     need = ulysses_workspace_bytes(P, S_l, H, D, out.dtype)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     _need_cuda(q, k, v, out, lse, workspace)
     st = lib().cpattn_ulysses_fwd_split(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), P, S_l,
                                         H, D, float(scale), _dtype_code(out.dtype),
-                                        _ptr(workspace),
-                                        workspace.numel() if workspace is not None else 0,
-                                        _stream(stream))
+                                        _ptr(workspace), _nbytes(workspace), _stream(stream))
     _check(st, "cpattn_ulysses_fwd_split")
     return out, lse
 
@@ -256,6 +275,10 @@ def fwd_split(q, k, v, out=None, lse=None, scale=None, out_dtype=None, accumulat
         out = torch.empty((B_, Sq, H, D), dtype=out_dtype or q.dtype, device=q.device)
     if lse is None:
         lse = torch.empty((B_, H, Sq), dtype=torch.float32, device=q.device)
+    if k.shape != (B_, Skv, H, D) or v.shape != (B_, Skv, H, D):
+        raise ValueError("k and v must be [B][Skv][H][D] matching q")
+    _need_shape(out, (B_, Sq, H, D), "out")
+    _need_shape(lse, (B_, H, Sq), "lse", torch.float32)
     if n_split is None:
         n_split = split_suggest(B_, H, Sq, Skv)
     need = split_workspace_bytes(B_, H, Sq, D, n_split, out.dtype, Skv=Skv)
@@ -264,7 +287,7 @@ def fwd_split(q, k, v, out=None, lse=None, scale=None, out_dtype=None, accumulat
     _need_cuda(q, k, v, out, lse, workspace)
     st = lib().cpattn_fwd_split(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B_, H, Sq, Skv,
                                 D, float(scale), _dtype_code(out.dtype), 1 if accumulate else 0,
-                                int(n_split), _ptr(workspace), workspace.numel(),
+                                int(n_split), _ptr(workspace), _nbytes(workspace),
                                 _stream(stream))
     _check(st, "cpattn_fwd_split")
     return out, lse
@@ -279,6 +302,7 @@ def fwd_accumulate(q, k, v, o_acc, lse_acc, scale=None, stream=None):
         raise ValueError("k and v must be [B][Skv][H][D] matching q")
     if o_acc.shape != (B, Sq, H, D) or lse_acc.shape != (B, H, Sq):
         raise ValueError("o_acc must be [B][Sq][H][D] and lse_acc [B][H][Sq]")
+    _need_shape(lse_acc, (B, H, Sq), "lse_acc", torch.float32)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     _need_cuda(q, k, v, o_acc, lse_acc)
@@ -296,6 +320,10 @@ def merge(o_a, lse_a, o_b, lse_b, out=None, lse=None, stream=None):
         out = torch.empty_like(o_a)
     if lse is None:
         lse = torch.empty_like(lse_a)
+    _need_shape(o_b, (B, S, H, D), "o_b", o_a.dtype)
+    _need_shape(out, (B, S, H, D), "out", o_a.dtype)
+    for name, t in (("lse_a", lse_a), ("lse_b", lse_b), ("lse", lse)):
+        _need_shape(t, (B, H, S), name, torch.float32)
     _need_cuda(o_a, lse_a, o_b, lse_b, out, lse)
     st = lib().cpattn_merge(_ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b), _ptr(out), _ptr(lse),
                             B, H, S, D, _dtype_code(o_a.dtype), _stream(stream))
@@ -310,6 +338,7 @@ def seq2head(src, P, out=None, stream=None):
         raise ValueError("src.shape[0] must equal P")
     if out is None:
         out = torch.empty((P, P * S_l, H // P, D), dtype=src.dtype, device=src.device)
+    _need_shape(out, (P, P * S_l, H // P, D), "out", src.dtype)
     _need_cuda(src, out)
     st = lib().cpattn_seq2head(_ptr(src), _ptr(out), P, S_l, H, D, src.element_size(),
                                _stream(stream))
@@ -325,6 +354,8 @@ def seq2head_qkv(q, k, v, P, out=None, stream=None):
     if out is None:
         out = tuple(torch.empty((P, P * S_l, H // P, D), dtype=q.dtype, device=q.device)
                     for _ in range(3))
+    for i, t in enumerate(out):
+        _need_shape(t, (P, P * S_l, H // P, D), f"out[{i}]", q.dtype)
     _need_cuda(q, k, v, *out)
     st = lib().cpattn_seq2head_qkv(_ptr(q), _ptr(k), _ptr(v), *(_ptr(t) for t in out), P, S_l, H,
                                    D, q.element_size(), _stream(stream))
@@ -363,6 +394,8 @@ def seq2head_qkv_norm(q, k, v, P, gamma_q, gamma_k, eps=1e-6, out_scale=1.0, out
     if out is None:
         out = tuple(torch.empty((P, P * S_l, H // P, D), dtype=q.dtype, device=q.device)
                     for _ in range(3))
+    for i, t in enumerate(out):
+        _need_shape(t, (P, P * S_l, H // P, D), f"out[{i}]", q.dtype)
     _need_cuda(q, k, v, gamma_q, gamma_k, *out)
     st = lib().cpattn_seq2head_qkv_norm(_ptr(q), _ptr(k), _ptr(v), *(_ptr(t) for t in out),
                                         _ptr(gamma_q), _ptr(gamma_k), P, S_l, H, D, float(eps),
@@ -379,6 +412,7 @@ def head2seq(src, P, out=None, stream=None):
     S_l, H = S_full // P, Hp * P
     if out is None:
         out = torch.empty((P, S_l, H, D), dtype=src.dtype, device=src.device)
+    _need_shape(out, (P, S_l, H, D), "out", src.dtype)
     _need_cuda(src, out)
     st = lib().cpattn_head2seq(_ptr(src), _ptr(out), P, S_l, H, D, src.element_size(),
                                _stream(stream))
