@@ -153,6 +153,11 @@ class UlyssesStreamer:
     def submit(self, hq, hk, hv, h_out, h_lse, scale=None):
         k = self.step % self.depth
         plan, (dq, dk, dv) = self.plans[k], self.inputs[k]
+        if any(t.shape != dq.shape for t in (hq, hk, hv)):
+            raise ValueError(f"host Q/K/V shards must be {tuple(dq.shape)}")
+        if h_out.shape != plan.out.shape or h_lse.shape != plan.lse.shape:
+            raise ValueError(f"h_out must be {tuple(plan.out.shape)} and h_lse "
+                             f"{tuple(plan.lse.shape)}")
         # waiting on an event that was never recorded returns at once (first rotation)
         self.upload.wait_event(self.computed[k])
         with torch.cuda.stream(self.upload):
