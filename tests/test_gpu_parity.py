@@ -544,10 +544,11 @@ def test_fused_ulysses_tail_split_full_size():
 
 @pytest.mark.parametrize("n_chunks", [1, 2, 3, 4])
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
-def test_ulysses_host_pass_equals_device_path(n_chunks, out_dtype):
+@pytest.mark.parametrize("D", [128, 64])
+def test_ulysses_host_pass_equals_device_path(n_chunks, out_dtype, D):
     # host shards in, host O/LSE out, copies pipelined over head-group chunks inside the
     # C-ABI call: the same bits as the device-resident fused call, and the oracle's values
-    P, S_l, H, D = 4, 400, 8, 128
+    P, S_l, H = 4, 400, 8
     g = torch.Generator().manual_seed(900 + n_chunks)
     host = [W.randn((P, S_l, H, D), g, 1.0, "bf16").pin_memory() for _ in range(3)]
     h_out = torch.full((P, S_l, H, D), float("nan"), dtype=out_dtype).pin_memory()
