@@ -340,6 +340,37 @@ def test_tail_split_matches_oracle(shape, out_dtype):
     assert (o_a.float() - o_t.float()).abs().max().item() < tol
 
 
+def test_tail_split_without_a_plan_needs_no_workspace():
+    # 3 key blocks: no range pays off, so the tail split is the single pass and takes a NULL
+    # workspace (the header allows it when nothing is split); bits equal to cpattn_fwd
+    import ctypes
+
+    Bn, H, Sq, Skv, D = 1, 4, 700, 300, 128
+    q, k, v = (t.to(DEV) for t in W.random_case(77, Bn, H, Sq, Skv, D))
+    assert cp.split_workspace_bytes(Bn, H, Sq, D, 0, torch.bfloat16, Skv=Skv) == 0
+    o1, l1 = cp.fwd(q, k, v)
+    o2, l2 = torch.empty_like(o1), torch.empty_like(l1)
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    st = cp.lib().cpattn_fwd_split(p(q), p(k), p(v), p(o2), p(l2), Bn, H, Sq, Skv, D,
+                                   1 / math.sqrt(D), 0, 0, 0, None, 0,
+                                   ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_fused_ulysses_split_single_rank():
+    # P = 1: no re-partition; 16 heads x 37 tile pairs = 592 items fill 4 waves exactly, so
+    # nothing is split and the call equals cpattn_ulysses_fwd bit for bit
+    g = torch.Generator().manual_seed(31)
+    s = [W.randn((1, 9472, 16, 64), g, 1.0, "bf16").to(DEV) for _ in range(3)]
+    assert cp.ulysses_workspace_bytes(1, 9472, 16, 64) == 0
+    o1, l1 = cp.ulysses_fwd(*s, 1)
+    o2, l2 = cp.ulysses_fwd_split(*s, 1)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
 def test_ring_step_with_tail_split():
     # one rank's ring step: 352 items on 148 SMs leave 56 in the last wave, split in two
     w = W.WORKLOADS[3]
